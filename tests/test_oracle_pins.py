@@ -1,0 +1,362 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a hand-derived value
+stored under tests/golden/ (with its derivation and page citation), a closed form, an
+invariant, a special case that reduces to a textbook routine, or brute force on tiny
+inputs.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import softmax
+
+from oracle import csa_oracle as O
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------- rounding
+
+def test_bf16_rounding_matches_known_values():
+    # 1 + 2^-8 is a tie between 1 and 1 + 2^-7 -> even mantissa (1.0); 1 + 3*2^-8 -> 1 + 2^-6.
+    assert O.bf16(1.0 + 2.0 ** -8) == 1.0
+    assert O.bf16(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert O.bf16(-2.0 ** -130) == -2.0 ** -130          # subnormal in bf16 is exact here
+    assert O.bf16(np.inf) == np.inf and np.isnan(O.bf16(np.nan))
+    # Every bf16 value round-trips.
+    bits = np.arange(0, 1 << 16, 7, dtype=np.uint32) << 16
+    vals = bits.view(np.float32).astype(np.float64)
+    fin = np.isfinite(vals)
+    assert np.array_equal(O.bf16(vals[fin]), vals[fin])
+
+
+# ----------------------------------------------------------------------------- RoPE (T8)
+
+def test_rope_matches_complex_rotation():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal(512)
+    pos, base, rd = 32767, 10000.0, 64
+    y = O.rope(x, pos, rd, base)
+    z = x[-rd:][0::2] + 1j * x[-rd:][1::2]
+    theta = np.array([base ** (-(2.0 * i) / rd) for i in range(rd // 2)])
+    zr = z * np.exp(1j * pos * theta)
+    assert np.allclose(y[-rd:][0::2], zr.real, atol=1e-12)
+    assert np.allclose(y[-rd:][1::2], zr.imag, atol=1e-12)
+    assert np.array_equal(y[:-rd], x[:-rd])
+
+
+def test_rope_inverse_identity_norm_and_position_zero():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((3, 512))
+    for pos in (0, 1, 127, 32767, 1048575):
+        y = O.rope(x, pos, 64, 10000.0)
+        assert np.allclose(O.rope(y, pos, 64, 10000.0, inverse=True), x, atol=1e-12)
+        assert np.allclose(np.linalg.norm(y[:, -64:], axis=1), np.linalg.norm(x[:, -64:], axis=1))
+    assert np.array_equal(O.rope(x, 0, 64, 10000.0), x)
+    # pair 0 has theta = 1: rotation by exactly pos radians
+    e = np.zeros(512); e[448] = 1.0
+    y = O.rope(e, 5, 64, 10000.0)
+    assert np.isclose(y[448], math.cos(5)) and np.isclose(y[449], math.sin(5))
+
+
+def test_entry_norm_rope_golden(golden_dir):
+    g = _load(golden_dir, "entry_norm_rope_hand.json")
+    y = O.finish_entry(np.array(g["x"]), g["g"], g["ratio"], 1.0, 0.0, 2, 10000.0)
+    assert np.allclose(y, g["expected"], atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- compressor
+
+def test_first_group_hand_example(golden_dir):
+    """T2: the first group pools only its 4 current slots; the -inf previous slots have weight 0."""
+    g = _load(golden_dir, "compress_first_group_hand.json")
+    prev_sc = np.full((4, 1), -np.inf)
+    prev_kv = np.full((4, 1), np.nan)          # never touched: skipped, not multiplied by 0
+    slot_kv = np.concatenate([prev_kv, np.array(g["cur_kv"])[:, None]])
+    slot_sc = np.concatenate([prev_sc, np.array(g["cur_scores"])[:, None]])
+    pooled, wts = O.pool_slots(slot_kv, slot_sc)
+    assert np.isclose(pooled[0], g["pooled"], atol=1e-12)
+    assert np.allclose(wts[4:, 0], g["weights"], atol=1e-12)
+    assert np.array_equal(wts[:4, 0], np.zeros(4))
+
+
+def test_first_group_reduces_to_four_slot_softmax():
+    rng = np.random.default_rng(3)
+    cfg = O.CompressorCfg(4, 16, rope_dim=8)
+    kv = rng.standard_normal((4, 32))
+    sc = rng.standard_normal((4, 32)) * 3
+    skv, ssc = O.init_state(cfg)
+    out = O.compress_tokens(cfg, skv, ssc, 0, kv, sc, np.ones(16))
+    w = softmax(sc[:, 16:], axis=0)
+    pooled = np.sum(w * kv[:, 16:], axis=0)
+    ref = O.rope(O.rms_norm(pooled, 1.0, cfg.eps), 0, 8, 10000.0)
+    assert np.allclose(out[0], ref, atol=1e-12)
+
+
+def test_weights_sum_to_one_and_constant_vector_closed_form():
+    """T1: per-channel weights sum to 1, so equal kv slots give RoPE(RMSNorm(v)) for any scores."""
+    rng = np.random.default_rng(4)
+    d = 512
+    v = rng.standard_normal(d)
+    gamma = 1 + 0.1 * rng.standard_normal(d)
+    cfg = O.CompressorCfg(4, d)
+    for trial in range(3):
+        sc = rng.standard_normal((8, 2 * d)) * 5
+        kv = np.tile(np.concatenate([v, v]), (8, 1))
+        out = O.compress_parallel(cfg, kv, sc, gamma)
+        _, wts = O.pool_slots(np.concatenate([kv[:4, :d], kv[4:, d:]]), np.concatenate([sc[:4, :d], sc[4:, d:]]))
+        assert np.allclose(wts.sum(axis=0), 1.0, atol=1e-12)
+        ref = O.rope(gamma * v / math.sqrt(np.mean(v * v) + 1e-6), 4, 64, 10000.0)
+        assert np.allclose(out[1], ref, atol=1e-10)
+
+
+def test_halves_come_from_previous_first_and_current_second():
+    """R1 (the torch.cat line of the C4A section): entry g mixes channels [:d] of the previous
+    group's tokens with channels [d:] of the current group's. Values placed in the other
+    halves must not appear; the result is a closed form in the two constant blocks."""
+    d = 8
+    cfg = O.CompressorCfg(4, d, rope_dim=2)
+    A, Bv, s1, s2 = 2.0, -3.0, 0.7, -0.4
+    kv = np.zeros((8, 2 * d)); sc = np.zeros((8, 2 * d))
+    kv[:4, :d] = A; kv[:4, d:] = 1e6          # previous group: first half A, second half junk
+    kv[4:, d:] = Bv; kv[4:, :d] = -1e6        # current group: second half B, first half junk
+    sc[:4, :d] = s1; sc[4:, d:] = s2
+    sc[:4, d:] = 50.0; sc[4:, :d] = 50.0      # junk scores must be ignored too
+    out = O.compress_parallel(cfg, kv, sc, np.ones(d))
+    pooled = (math.exp(s1) * A + math.exp(s2) * Bv) / (math.exp(s1) + math.exp(s2))
+    x = np.full(d, pooled)
+    ref = O.rope(x / math.sqrt(pooled * pooled + 1e-6), 4, 2, 10000.0)
+    assert np.allclose(out[1], ref, atol=1e-9)
+
+
+@pytest.mark.parametrize("ratio,d", [(4, 64), (4, 128), (128, 64)])
+def test_state_machine_equals_parallel_and_chunked(ratio, d):
+    """T3: the token-by-token rolling state equals the direct per-group formula, and
+    uneven chunks resumed from the state equal one shot."""
+    rng = np.random.default_rng(5 + ratio)
+    cfg = O.CompressorCfg(ratio, d)
+    S = 8 * ratio + 3
+    kv = rng.standard_normal((S, cfg.width))
+    sc = rng.standard_normal((S, cfg.width)) * 2
+    gamma = 1 + 0.1 * rng.standard_normal(d)
+    par = O.compress_parallel(cfg, kv, sc, gamma)
+    skv, ssc = O.init_state(cfg)
+    seq = O.compress_tokens(cfg, skv, ssc, 0, kv, sc, gamma)
+    assert sorted(seq) == list(range(S // ratio))
+    for g in seq:
+        assert np.allclose(seq[g], par[g], atol=1e-12)
+    # chunked: uneven splits
+    cuts = [0, 1, ratio + 2, 3 * ratio - 1, 5 * ratio, S]
+    skv2, ssc2 = O.init_state(cfg)
+    got = {}
+    for lo, hi in zip(cuts[:-1], cuts[1:]):
+        got.update(O.compress_tokens(cfg, skv2, ssc2, lo, kv[lo:hi], sc[lo:hi], gamma))
+    assert sorted(got) == sorted(seq)
+    for g in got:
+        assert np.array_equal(got[g], seq[g])
+    assert np.array_equal(skv2, skv) and np.array_equal(ssc2, ssc)
+
+
+def test_entry_visible_only_when_group_completes():
+    """T4 (compressor side): entry g is emitted at t = ratio*g + ratio - 1 and not before."""
+    cfg = O.CompressorCfg(4, 16, rope_dim=8)
+    rng = np.random.default_rng(6)
+    skv, ssc = O.init_state(cfg)
+    for t in range(20):
+        res = O.compressor_step(cfg, skv, ssc, t, rng.standard_normal(32), rng.standard_normal(32), 1.0)
+        if (t + 1) % 4 == 0:
+            assert res is not None and res[0] == t // 4
+        else:
+            assert res is None
+        assert O.visible_entries(t, 4) == (t + 1) // 4
+
+
+# ----------------------------------------------------------------------------- indexer / top-k
+
+def test_indexer_hand_example(golden_dir):
+    g = _load(golden_dir, "indexer_hand.json")
+    s = O.indexer_scores(np.array(g["q_idx"]), np.array(g["w"]), np.array(g["idx_cache"]), 3)
+    assert np.allclose(s, g["expected"], atol=1e-15)
+    s2 = O.indexer_scores(np.array(g["q_idx"]), np.array(g["w"]), np.array(g["idx_cache"]), 2)
+    assert s2.shape == (2,)
+
+
+def test_indexer_brute_force_loops():
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((3, 5)); w = rng.standard_normal(3); k = rng.standard_normal((6, 5))
+    s = O.indexer_scores(q, w, k, 6)
+    for j in range(6):
+        acc = 0.0
+        for h in range(3):
+            dot = sum(q[h, c] * k[j, c] for c in range(5))
+            acc += w[h] * (dot if dot > 0 else 0.0)
+        assert abs(acc - s[j]) < 1e-12
+
+
+def _beats(a, b, sc):
+    """Total order of the selection: higher score first, lower index on ties."""
+    return sc[a] > sc[b] or (sc[a] == sc[b] and a < b)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_brute_force_over_all_subsets(seed):
+    rng = np.random.default_rng(100 + seed)
+    n, k = 8, 3
+    sc = rng.integers(-3, 4, size=n).astype(np.float64)    # many ties
+    if seed == 0:
+        sc[:] = 0.0
+        sc[[1, 5]] = -0.0
+    sel = O.topk_select(sc, k)
+    winners = [set(c) for c in itertools.combinations(range(n), k)
+               if all(_beats(a, b, sc) for a in c for b in range(n) if b not in c)]
+    assert len(winners) == 1
+    assert set(sel.tolist()) == winners[0]
+    assert list(sel) == sorted(sel)
+
+
+def test_topk_padding_and_nan():
+    sel = O.topk_select(np.array([0.5, 2.0, -1.0]), 5)
+    assert sel.tolist() == [0, 1, 2, -1, -1]
+    sel = O.topk_select(np.array([np.nan, 1.0, 0.0, np.nan]), 2)
+    assert sel.tolist() == [1, 2]
+    sel = O.topk_select(np.array([]), 3)
+    assert sel.tolist() == [-1, -1, -1]
+
+
+# ----------------------------------------------------------------------------- attention
+
+def test_sink_softmax_hand_example(golden_dir):
+    g = _load(golden_dir, "sink_softmax_hand.json")
+    o = O.mqa_with_sink(np.array([g["q"]]), np.array(g["cand"]), np.array([g["sink"]]), 1.0)
+    assert np.allclose(o[0], g["expected"], atol=1e-12)
+
+
+def test_sink_to_minus_infinity_is_plain_softmax():
+    """T6."""
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((4, 16)); c = rng.standard_normal((9, 16))
+    o = O.mqa_with_sink(q, c, np.full(4, -np.inf), 0.25)
+    ref = softmax(0.25 * q @ c.T, axis=1) @ c
+    assert np.allclose(o, ref, atol=1e-12)
+
+
+def test_sink_equals_extra_zero_value_column():
+    rng = np.random.default_rng(9)
+    q = rng.standard_normal((4, 16)); c = rng.standard_normal((9, 16)); sink = rng.standard_normal(4) * 3
+    o = O.mqa_with_sink(q, c, sink, 0.25)
+    logits = np.concatenate([0.25 * q @ c.T, sink[:, None]], axis=1)
+    vals = np.concatenate([c, np.zeros((1, 16))], axis=0)
+    assert np.allclose(o, softmax(logits, axis=1) @ vals, atol=1e-12)
+
+
+def test_window_positions():
+    assert O.window_positions(5, 16) == list(range(0, 6))
+    assert O.window_positions(100, 16) == list(range(85, 101))
+    assert O.window_positions(0, 128) == [0]
+
+
+def _dense_reference(q, t, W, ring, ring_cap, cache, n_vis, sink, scale, rope_dim, base):
+    """Textbook softmax attention over window + every visible entry, with the sink as an
+    extra logit carrying a zero value row, then the inverse rotation by t written with
+    complex numbers."""
+    rows = [ring[p % ring_cap] for p in range(max(0, t - W + 1), t + 1)] + [cache[s] for s in range(n_vis)]
+    C = np.array(rows)
+    logits = np.concatenate([scale * q @ C.T, sink[:, None]], axis=1)
+    o = softmax(logits, axis=1) @ np.concatenate([C, np.zeros((1, C.shape[1]))])
+    z = o[:, -rope_dim:][:, 0::2] + 1j * o[:, -rope_dim:][:, 1::2]
+    theta = np.array([base ** (-(2.0 * i) / rope_dim) for i in range(rope_dim // 2)])
+    z = z * np.exp(-1j * t * theta)
+    o[:, -rope_dim:][:, 0::2] = z.real
+    o[:, -rope_dim:][:, 1::2] = z.imag
+    return o
+
+
+def test_topk_at_least_visible_reduces_to_dense_attention():
+    """T5 on the tiny shape (8 heads x 512, window 16, ratio 4): with k >= visible the CSA
+    layer is dense attention over window + all entries."""
+    rng = np.random.default_rng(10)
+    S, H, d, W = 128, 8, 512, 16
+    inp = dict(
+        kv=rng.standard_normal((1, S, 2 * d)), score=rng.standard_normal((1, S, 2 * d)),
+        idx_kv=rng.standard_normal((1, S, 256)), idx_score=rng.standard_normal((1, S, 256)),
+        win_kv=rng.standard_normal((1, S, d)), q=rng.standard_normal((1, S, H, d)) / math.sqrt(d) * 3,
+        q_idx=rng.standard_normal((1, S, 4, 128)), w=rng.standard_normal((1, S, 4)),
+        sink=rng.standard_normal(H), gamma=np.ones(d), idx_gamma=np.ones(128),
+        pos=np.arange(S)[None, :])
+    qs = [0, 3, 4, 17, 64, 127]
+    res = O.csa_prefill(inp, 0, qs, H=H, d=d, W=W, topk=S // 4)
+    for i in qs:
+        ref = _dense_reference(inp["q"][0, i], i, W, inp["win_kv"][0], S, res["cache"], (i + 1) // 4,
+                               inp["sink"], 1 / math.sqrt(d), 64, 10000.0)
+        assert np.allclose(res["queries"][i]["out"], ref, atol=1e-10)
+
+
+def test_future_group_values_do_not_leak():
+    """T4: adversarial values in an incomplete group (and later tokens) do not change the
+    output of any query that precedes the group's completion."""
+    rng = np.random.default_rng(11)
+    S, H, d, W = 64, 4, 512, 16
+    base = dict(
+        kv=rng.standard_normal((1, S, 2 * d)), score=rng.standard_normal((1, S, 2 * d)),
+        idx_kv=rng.standard_normal((1, S, 256)), idx_score=rng.standard_normal((1, S, 256)),
+        win_kv=rng.standard_normal((1, S, d)), q=rng.standard_normal((1, S, H, d)) / 8,
+        q_idx=rng.standard_normal((1, S, 4, 128)), w=rng.standard_normal((1, S, 4)),
+        sink=rng.standard_normal(H), gamma=np.ones(d), idx_gamma=np.ones(128), pos=np.arange(S)[None, :])
+    t_query = 41                      # group 10 = tokens 40..43 is incomplete at t = 41
+    bad = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in base.items()}
+    for key in ("kv", "score", "idx_kv", "idx_score"):
+        bad[key][0, 42:] = 1e4
+    bad["win_kv"][0, 42:] = 1e4
+    a = O.csa_prefill(base, 0, [t_query], H=H, d=d, W=W, topk=4)
+    b = O.csa_prefill(bad, 0, [t_query], H=H, d=d, W=W, topk=4)
+    assert np.array_equal(a["queries"][t_query]["out"], b["queries"][t_query]["out"])
+    # ... while a query after completion does see the change.
+    a = O.csa_prefill(base, 0, [47], H=H, d=d, W=W, topk=4)
+    b = O.csa_prefill(bad, 0, [47], H=H, d=d, W=W, topk=4)
+    assert not np.allclose(a["queries"][47]["out"], b["queries"][47]["out"])
+
+
+# ----------------------------------------------------------------------------- counters (T7)
+
+def test_flop_ledger_matches_printed_values(golden_dir):
+    g = _load(golden_dir, "flop_ledger.json")
+    c, h = g["csa"], g["hca"]
+    rc = O.reads_per_query(c["t"], c["window"], c["ratio"], c["topk"])
+    rh = O.reads_per_query(h["t"], h["window"], h["ratio"], None)
+    assert rc == c["reads"] and rh == h["reads"]
+    fc = O.attention_flops(g["heads"], rc, g["d"])
+    fh = O.attention_flops(g["heads"], rh, g["d"])
+    assert fc == c["flops"] and fh == h["flops"]
+    assert round(fc / 1e6) == c["printed_mflop"] and round(fh / 1e6) == h["printed_mflop"]
+
+
+def test_reads_per_query_edge_cases():
+    assert O.reads_per_query(0, 128, 4, 1024) == 1          # first token: itself only
+    assert O.reads_per_query(3, 128, 4, 1024) == 5          # entry 0 completes at t = 3
+    assert O.reads_per_query(8191, 128, 4, 1024) == 128 + 1024
+    assert O.reads_per_query(1048575, 128, 4, 1024) == 1152
+
+
+def test_large_sink_stays_finite():
+    """R6: the running max includes the sink, so a sink far above every logit gives an
+    output near zero instead of overflowing."""
+    q = np.ones((1, 4)); c = np.ones((3, 4)) * 0.1
+    o = O.mqa_with_sink(q, c, np.array([1000.0]), 1.0)
+    assert np.all(np.isfinite(o)) and np.max(np.abs(o)) < 1e-300
+
+
+def test_rmsnorm_eps_matters_for_small_vectors():
+    """R3: eps = 1e-6 sits inside the square root. For a constant vector of 1e-4 the
+    normalised value is 1e-4 / sqrt(1e-8 + 1e-6); a zero vector stays zero."""
+    x = np.full(8, 1e-4)
+    y = O.rms_norm(x, 1.0, 1e-6)
+    assert np.allclose(y, 1e-4 / math.sqrt(1e-8 + 1e-6), rtol=1e-12)
+    assert np.array_equal(O.rms_norm(np.zeros(8), 1.0, 1e-6), np.zeros(8))
