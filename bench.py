@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA layer on B200: prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Default workload: Pro CSA decode, B=64 requests per GPU at 32K context (8192 compressed entries,
+128-token window, 128 heads x 512, indexer 64 x 128, top-k 1024). A step is one fused decode
+step of every request through the C ABI (compressor step of the main and index streams + window
+write, indexer, top-k, sparse MQA with sink, inverse RoPE). Inputs are synthetic, resident in
+HBM, and rotate over several sets whose per-step footprint exceeds the 126 MB L2, so no step is
+served from data the previous step left in L2. Multi-GPU runs shard requests (each rank owns its
+own B requests; no collective on the data path) and report the whole-job aggregate.
+
+--impl reference times the CPU oracle (the plain float64 reference of the layer) on the host
+cores, on a bounded sample of the same workload, as the reference arm.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from synth import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "CSA decode queries/s @32K ctx B=64; achieved HBM GB/s as % of B200 peak"
+
+
+# ------------------------------------------------------------------------------ helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernel_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "long_context_decode_c4a_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str, files):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_hash") != kernel_hash(files):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------ per-step byte / flop ledgers
+
+def decode_bytes(wl):
+    """Algorithmic HBM bytes per query of each kernel of one CSA/HCA decode step."""
+    E = wl.max_entries
+    reads = wl.W + (min(wl.topk, E) if wl.has_indexer else E)
+    width = (1 + wl.overlap) * wl.d
+    rows = (1 + wl.overlap) * wl.ratio
+    out = {}
+    # compressor step: state rows (kv + score) read, the token's streams read, state row(s) written,
+    # the entry written; window row read + written.
+    comp = 2 * rows * width * 2 + 2 * width * 2 + wl.d * 2 + 2 * wl.d * 2
+    if wl.has_indexer:
+        comp += 2 * 8 * 2 * wl.d_I * 2 + 2 * 2 * wl.d_I * 2 + wl.d_I * 2
+        out["indexer"] = E * wl.d_I * 2 + wl.H_I * wl.d_I * 2 + wl.H_I * 4 + E * 4
+        out["topk"] = E * 4 + wl.topk * 4
+    out["compress"] = comp
+    out["attention"] = reads * wl.d * 2 + 2 * wl.H * wl.d * 2 + (wl.topk * 4 if wl.has_indexer else 0)
+    return out, reads
+
+
+# ------------------------------------------------------------------------------ our arm
+
+def step_inputs(inp):
+    keys = ["pos", "kv", "score", "idx_kv", "idx_score", "win_kv", "q", "q_idx", "w"]
+    return {k: inp[k][:, 0].contiguous() if inp[k].dim() > 1 and k != "pos" else inp[k][:, 0].contiguous()
+            for k in keys if k in inp}
+
+
+def run_ours_decode(wl, args, world, rank):
+    from long_context_decode_c4a_b200 import ops
+    dev = torch.device("cuda")
+    csa = wl.has_indexer
+    sets = []
+    for s in range(args.sets):
+        inp = make_inputs(wl, device="cuda", seed=wl.seed + 1000 * rank + s)
+        if csa:
+            st = ops.CsaDecodeState(wl.B, wl.max_entries, H=wl.H, d=wl.d, H_I=wl.H_I, d_I=wl.d_I, window=wl.W,
+                                    topk=wl.topk, device=dev)
+            names = ("state_kv", "state_score", "idx_state_kv", "idx_state_score", "cache", "idx_cache", "ring")
+        else:
+            st = ops.HcaDecodeState(wl.B, wl.max_entries, H=wl.H, d=wl.d, window=wl.W, ratio=wl.ratio, device=dev)
+            names = ("state_kv", "state_score", "cache", "ring")
+        for n in names:
+            getattr(st, n).copy_(inp[n])
+        x = step_inputs(inp)
+        x["sink"] = inp["sink"]
+        x["out"] = torch.empty(wl.B, wl.H, wl.d, dtype=torch.bfloat16, device=dev)
+        sets.append((st, x))
+        del inp
+    torch.cuda.synchronize()
+
+    def call(st, x, evs=None):
+        if csa:
+            st.step(x["pos"], x["kv"], x["score"], x["idx_kv"], x["idx_score"], x["win_kv"], x["q"], x["q_idx"],
+                    x["w"], x["sink"], out=x["out"], stage_events=evs)
+        else:
+            st.step(x["pos"], x["kv"], x["score"], x["win_kv"], x["q"], x["sink"], out=x["out"], stage_events=evs)
+
+    nstage = 5 if csa else 3
+    for i in range(args.warmup):
+        call(*sets[i % len(sets)])
+    torch.cuda.synchronize()
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
+    for row in stage_ev:       # create the underlying events before the timed region
+        for e in row:
+            e.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device())
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record()
+    for k in range(args.steps):
+        call(*sets[k % len(sets)], evs=stage_ev[k])
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms, world)
+    for st, _ in sets:
+        status = ops.device_status(st.ws)
+        if status != 0:
+            raise RuntimeError(f"device status {status} after the timed steps")
+
+    stage_names = ["compress", "indexer", "topk", "attention"] if csa else ["compress", "attention"]
+    stage_ms = {n: statistics.mean(stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(args.steps))
+                for i, n in enumerate(stage_names)}
+
+    # ---- end-to-end through the public API with host buffers
+    st, x = sets[0]
+    host = {k: v.to("cpu").pin_memory() for k, v in x.items() if k not in ("out", "sink")}
+    out_host = torch.empty(x["out"].shape, dtype=x["out"].dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+
+    def e2e_step(i):
+        stt, xx = sets[i % len(sets)]
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        xin = dict(xx)
+        xin.update(dev_in)
+        call(stt, xin)
+        out_host.copy_(xin["out"], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for k in range(args.steps):
+        e2e_step(k)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    launches_per_step = (4 + (1 if wl.max_entries > 16384 else 0)) if csa else 2
+    return dict(ms=ms, stage_ms=stage_ms, clocks=clk, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
+                launches=launches_per_step * args.steps)
+
+
+def oracle_decode_time(wl, n_req: int, seed: int = 1):
+    """Seconds the CPU oracle takes for n_req requests of the decode workload."""
+    from oracle import csa_oracle as O
+    small = wl.scaled(B=n_req)
+    inp = O.to_numpy_inputs(make_inputs(small, seed=seed))
+    t = time.perf_counter()
+    for b in range(n_req):
+        if wl.has_indexer:
+            O.csa_decode_request(inp, b, H=wl.H, d=wl.d, W=wl.W, topk=wl.topk)
+        else:
+            O.hca_decode_request(inp, b, H=wl.H, d=wl.d, W=wl.W, ratio=wl.ratio)
+    return time.perf_counter() - t
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def cpu_baseline_decode(wl, budget_s: float = 15.0):
+    one = oracle_decode_time(wl, 1)
+    n = int(max(1, min(wl.B, budget_s / max(one, 1e-3))))
+    secs = oracle_decode_time(wl, n, seed=2)
+    return {"value": n / secs, "unit": "queries/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n} of the {wl.B} requests of one step ({wl.name}), float64 numpy oracle"}
+
+
+# ------------------------------------------------------------------------------ main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="pro_csa_decode_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--sets", type=int, default=4, help="rotating input sets")
+    ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = WORKLOADS[args.workload]
+    if args.batch:
+        wl = wl.scaled(B=args.batch)
+    if not wl.is_decode:
+        ap.error("bench.py times the decode workloads; prefill has its own benchmark in the test suite")
+
+    if args.impl == "reference":
+        return run_reference(wl, args)
+
+    world, rank, local = dist_setup(args.gpus)
+    r = run_ours_decode(wl, args, world, rank)
+    peaks = load_peaks()
+    per_q, reads = decode_bytes(wl)
+    B_total = wl.B * world
+    value = B_total * 1000.0 / r["ms"]
+    # dominant kernel (largest share of the step) and its roofline
+    dom = max(("indexer", "attention") if wl.has_indexer else ("attention",), key=lambda n: r["stage_ms"][n])
+    bytes_launch = per_q[dom] * wl.B
+    achieved = bytes_launch / (r["stage_ms"][dom] * 1e-3) / 1e9
+    files = {"indexer": ["indexer.cu", "ptx.cuh", "kernels.cuh"],
+             "attention": ["attn.cu", "ptx.cuh", "kernels.cuh"]}[dom]
+    total_bytes = sum(per_q.values()) * wl.B
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": r["ms"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "global_batch": B_total, "requests_per_gpu": wl.B, "context": wl.ctx,
+                   "compressed_entries": wl.max_entries, "window": wl.W, "heads": wl.H, "head_dim": wl.d,
+                   "indexer_heads": wl.H_I, "topk": wl.topk, "reads_per_query": reads,
+                   "parallelism": f"requests sharded over {world} GPU(s), no data-path collective",
+                   "l2": f"{args.sets} rotating input sets, each step reads {total_bytes / 1e6:.0f} MB > 126 MB L2"},
+        "tokens_per_s": value,
+        "step_hbm_gbs": total_bytes / (r["ms"] * 1e-3) / 1e9,
+        "step_hbm_frac": total_bytes / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "kernels_ms": r["stage_ms"],
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "traffic": traffic_for(dom, wl.name, files),
+                     "algorithmic_bytes_per_launch": bytes_launch},
+        "e2e": {"value": B_total * 1000.0 / r["e2e_ms"], "unit": "queries/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"]},
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_decode(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def run_reference(wl, args):
+    """The reference arm: the CPU oracle as it stands, rank 0 only, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    one = oracle_decode_time(wl, 1)
+    per_step = max(1, min(wl.B, int(6.0 / max(one, 1e-3))))
+    total_steps = args.warmup + args.steps
+    while per_step > 1 and total_steps * per_step * one > 150:
+        per_step //= 2
+    for i in range(args.warmup):
+        oracle_decode_time(wl, per_step, seed=10 + i)
+    secs = [oracle_decode_time(wl, per_step, seed=100 + k) for k in range(args.steps)]
+    value = per_step * args.steps / sum(secs)
+    cores = cpu_threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * sum(secs) / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "global_batch": wl.B, "requests_per_gpu": wl.B, "context": wl.ctx,
+                   "sample_requests_per_step": per_step},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} requests of {wl.name} per step, float64 numpy oracle"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

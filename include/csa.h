@@ -1,0 +1,291 @@
+/*
+ * csa.h -- C ABI of libcsa.so: the DeepSeek-V4-Pro compressed-sparse-attention (CSA)
+ * layer and its heavily-compressed (HCA) variant on NVIDIA B200 (sm_100a).
+ *
+ * Sources, cited by page title and section:
+ *   [P1] "DeepSeek-V4-Pro 架构：一个 token 的旅程" (hs-black.github.io/posts/deepseek-v4-pro)
+ *   [P5] "图解DeepSeek V4：详细计算流程解析" (jsqmd.com)
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "dev" are device pointers owned by the caller. The library never
+ *     allocates or frees memory; scratch space is the caller's workspace `ws`.
+ *   - bf16 values are passed as uint16_t (IEEE bfloat16 bit patterns).
+ *   - `stream` is a cudaStream_t passed as void*. Every call only enqueues work on it; no
+ *     call synchronises the host except csa_get_device_status.
+ *   - Every call returns a csa_status. Arguments are checked on the host before any launch:
+ *     on CSA_ERR_INVALID_ARG / CSA_ERR_UNSUPPORTED / CSA_ERR_WORKSPACE nothing was enqueued.
+ *     CSA_ERR_CUDA reports a launch error; csa_last_error() gives its text.
+ *   - Device-side faults never trap: a kernel that gives up a bounded wait, or that meets an
+ *     out-of-range index, records a code in the workspace status word and returns.
+ *     csa_get_device_status reads it.
+ *   - Positions t are absolute token positions (0-based). Batch strides are in elements.
+ *   - Thread safety: the library keeps no state except a thread-local error string.
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA_API __attribute__((visibility("default")))
+#else
+#define CSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer or stride */
+  CSA_ERR_UNSUPPORTED = 2,   /* a shape outside what the kernels implement */
+  CSA_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  CSA_ERR_TIMEOUT = 4,       /* (device status) a bounded wait inside a kernel gave up */
+  CSA_ERR_WORKSPACE = 5,     /* ws is null, misaligned or smaller than csa_workspace_size */
+  CSA_ERR_BOUNDS = 6         /* (device status) an index read from memory was out of range */
+} csa_status;
+
+/* Text of a status code (static string). */
+CSA_API const char* csa_status_string(int status);
+/* Text of the last CSA_ERR_CUDA / argument error seen on the calling thread. */
+CSA_API const char* csa_last_error(void);
+/* ABI version: 1. */
+CSA_API int csa_version(void);
+
+/*
+ * Compressor configuration.
+ *   ratio 4,  overlap 1: C4A. Each token carries kv and score streams of width 2d; compressed
+ *             entry g pools channels [:d] of group g-1's 4 tokens and channels [d:] of group
+ *             g's 4 tokens (8 slots per channel) ([P5] §2.1, the torch.cat of pre/cur state).
+ *   ratio 128, overlap 0: C128A. Streams of width d; entry g pools tokens 128g..128g+127
+ *             ([P5] §3.1, "state is concatenated directly").
+ * Pooling is a per-channel softmax over the slots times kv, summed over slots; then
+ * RMSNorm (gamma, eps) over the d dims, then RoPE on the last rope_dim dims at position
+ * g*ratio ([P1] "压缩是逐通道的 learned pooling"). RoPE rotates adjacent pairs (2i, 2i+1) by
+ * pos * rope_base^(-2i/rope_dim).
+ * Supported: (ratio, overlap) in {(4,1), (128,0)}; d in {128, 512}; rope_dim 64 (even, <= d,
+ * multiple of 8).
+ */
+typedef struct {
+  int ratio;
+  int overlap;
+  int d;
+  int rope_dim;
+  float rope_base;
+  float eps;
+} csa_compressor_cfg;
+
+/* Workspace kinds for csa_workspace_size. */
+enum {
+  CSA_WS_INDEXER_TOPK = 1,
+  CSA_WS_SPARSE_ATTN = 2,
+  CSA_WS_HCA_ATTN = 3,
+  CSA_WS_DECODE_FUSED = 4,
+  CSA_WS_HCA_DECODE_FUSED = 5
+};
+
+/*
+ * Bytes of workspace the call of `kind` needs for B requests x S queries, with up to
+ * max_entries compressed entries per request and top-k `topk` (ignored for HCA kinds).
+ * The workspace must be 256-byte aligned. Its first 256 bytes hold the device status word;
+ * the caller zeroes the whole workspace once before first use (later calls keep the status
+ * word sticky until csa_get_device_status clears it).
+ */
+CSA_API int csa_workspace_size(int kind, int B, int S, int max_entries, int topk, size_t* bytes);
+
+/*
+ * Put a compressor state into its initial value: kv rows 0, score rows -inf, so that the
+ * previous-group slots of group 0 carry gate -inf and weight 0 ([P1] "一个通道，逐项算出压缩结果").
+ *   state_kv, state_score: dev bf16 [B, rows, width], rows = (1+overlap)*ratio,
+ *                          width = (1+overlap)*d.
+ */
+CSA_API int csa_state_reset(const csa_compressor_cfg* cfg, int B, uint16_t* state_kv, uint16_t* state_score,
+                    void* stream);
+
+/*
+ * csa_compress -- run the compressor over a segment of S new tokens per request
+ * ([P5] §2.1 and §3.1; [P1] "压缩条目必须等整组完成后才可见": entry t//ratio is written when
+ * (t+1) % ratio == 0; prefill computes every completed entry of the segment in parallel).
+ *   start_pos   dev int32 [B]: position of each request's first new token.
+ *   kv, score   dev bf16 [B, S, width] (width = (1+overlap)*d), contiguous.
+ *   gamma       dev bf16 [d]: RMSNorm weight.
+ *   state_kv, state_score  dev bf16 [B, rows, width], in/out. On entry: the state after token
+ *               start_pos-1 (or csa_state_reset). On exit: the state after token start_pos+S-1,
+ *               exactly as the token-by-token rolling state would leave it: token p lives in row
+ *               ratio + p%ratio (C4A) or p%ratio (C128A); after each completed group the C4A cur
+ *               rows are copied over the pre rows.
+ *   cache       dev bf16, entry g of request b at cache + b*cache_bstride + g*d. Only entries that
+ *               complete inside the segment are written. g must be < max_entries.
+ *   cache_f32   optional dev float with the same layout (nullable): the same entries before the
+ *               bf16 rounding.
+ * Alignment: all pointers 16-byte aligned; cache_bstride a multiple of 8.
+ * Errors: CSA_ERR_INVALID_ARG on a null or misaligned pointer, B<=0, S<=0.
+ */
+CSA_API int csa_compress(const csa_compressor_cfg* cfg, int B, int S, const int32_t* start_pos,
+                 const uint16_t* kv, const uint16_t* score, const uint16_t* gamma,
+                 uint16_t* state_kv, uint16_t* state_score,
+                 uint16_t* cache, int64_t cache_bstride, int max_entries, float* cache_f32,
+                 void* stream);
+
+/*
+ * csa_indexer_topk -- lightning indexer and top-k selection ([P1] "少读 KV 之前，Indexer 仍要给历史打分";
+ * [P5] §2.2). For query i of request b at position t = q_pos[b*S+i], with E = (t+1)//ratio visible
+ * entries:
+ *     score[s] = sum_h w[h] * ReLU(q_idx[h,:] . idx_cache[s,:])      for s < E
+ * then the indices of the min(topk, E) largest scores (ties to the lower index), written in
+ * ascending order and padded with -1.
+ *   q_pos     dev int32 [B, S].
+ *   q_idx     dev bf16 [B, S, H_I, d_I].   w: dev float [B, S, H_I] (may be negative).
+ *   idx_cache dev bf16, entry s of request b at idx_cache + b*idx_bstride + s*d_I.
+ *   topk_idx  dev int32 [B, S, topk], out.
+ *   scores_opt optional dev float [B, S, max_entries], out (nullable): the scores, s < E only.
+ *   ws/ws_bytes: workspace of at least csa_workspace_size(CSA_WS_INDEXER_TOPK, ...).
+ * Supported: d_I = 128; H_I a power of two <= 256; topk in [1, 2048]; E <= max_entries <= 2^24.
+ * A query with E > max_entries records CSA_ERR_BOUNDS in the status word and uses max_entries.
+ */
+CSA_API int csa_indexer_topk(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
+                     const uint16_t* q_idx, const float* w, const uint16_t* idx_cache,
+                     int64_t idx_bstride, int max_entries, int32_t* topk_idx, float* scores_opt,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * csa_sparse_attn -- sparse MQA over one candidate set with a learned sink, then inverse RoPE
+ * ([P1] "局部和压缩记忆，共用一次归一化" and "输出投影也分组"; [P5] §2 and §2.3).
+ * For query i of request b at position t:
+ *   candidates C = window rows ring[p % ring_cap] for p = max(0, t-window+1) .. t
+ *                  plus cache rows s for every topk_idx[b,i,j] >= 0 (entries < max_entries);
+ *   one cached row serves as key and value (MQA). For each head h:
+ *     l_j = scale * q[h] . c_j;  m = max(max_j l_j, sink[h]);
+ *     o[h] = sum_j e^(l_j-m) c_j / (sum_j e^(l_j-m) + e^(sink[h]-m));
+ *   then the last rope_dim dims of o[h] are rotated by -t (inverse RoPE).
+ *   q      dev bf16 [B, S, H, d].   sink: dev float [H].
+ *   ring   dev bf16, slot j of request b at ring + b*ring_bstride + j*d; window <= ring_cap.
+ *   cache  dev bf16, entry s at cache + b*cache_bstride + s*d.
+ *   topk_idx dev int32 [B, S, topk].
+ *   out    dev [B, S, H, d]: bf16 if out_is_f32 == 0, float otherwise.
+ * Supported: d = 512, rope_dim 64, 1 <= H <= 128, window <= 1024, topk <= 2048.
+ * Alignment: pointers 16 bytes; ring_bstride and cache_bstride multiples of d.
+ */
+CSA_API int csa_sparse_attn(int B, int S, int H, int d, int rope_dim, float rope_base, float scale,
+                    const int32_t* q_pos, const uint16_t* q, const uint16_t* ring,
+                    int64_t ring_bstride, int ring_cap, int window, const uint16_t* cache,
+                    int64_t cache_bstride, int max_entries, const int32_t* topk_idx, int topk,
+                    const float* sink, void* out, int out_is_f32, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
+ * hca_attn -- HCA attention ([P5] §3: no index module): as csa_sparse_attn, but the compressed
+ * candidates are every visible entry s < (t+1)//ratio (capped at max_entries), read in order.
+ * Supported: as csa_sparse_attn, with at most 2048 visible entries per query.
+ */
+CSA_API int hca_attn(int B, int S, int H, int d, int rope_dim, float rope_base, float scale, int ratio,
+             const int32_t* q_pos, const uint16_t* q, const uint16_t* ring, int64_t ring_bstride,
+             int ring_cap, int window, const uint16_t* cache, int64_t cache_bstride,
+             int max_entries, const float* sink, void* out, int out_is_f32, void* ws,
+             size_t ws_bytes, void* stream);
+
+/*
+ * Arguments of one CSA decode step for B requests (S = 1), each at its own position pos[b].
+ * Shapes follow [P5] §2: per token the main compressor streams are [2d], the index compressor
+ * streams [2 d_I], the window row [d] (already rotated by RoPE upstream), q [H, d], q_idx
+ * [H_I, d_I], w [H_I].
+ */
+typedef struct {
+  int B;
+  int H, d, rope_dim;          /* 128, 512, 64 */
+  int H_I, d_I;                /* 64, 128 */
+  int ratio;                   /* 4 */
+  int window;                  /* 128 */
+  int topk;                    /* 1024 */
+  float rope_base, eps, scale; /* 1e4, 1e-6, 1/sqrt(d) */
+  const int32_t* pos;          /* dev [B] */
+  const uint16_t* kv;          /* dev [B, 2d]   main compressor kv stream of token pos[b] */
+  const uint16_t* score;       /* dev [B, 2d] */
+  const uint16_t* idx_kv;      /* dev [B, 2d_I] index compressor streams */
+  const uint16_t* idx_score;   /* dev [B, 2d_I] */
+  const uint16_t* win_kv;      /* dev [B, d] window row of token pos[b] */
+  const uint16_t* q;           /* dev [B, H, d] */
+  const uint16_t* q_idx;       /* dev [B, H_I, d_I] */
+  const float* w;              /* dev [B, H_I] */
+  const float* sink;           /* dev [H] */
+  const uint16_t* gamma;       /* dev [d] */
+  const uint16_t* idx_gamma;   /* dev [d_I] */
+  uint16_t* state_kv;          /* dev [B, 2ratio, 2d] in/out */
+  uint16_t* state_score;
+  uint16_t* idx_state_kv;      /* dev [B, 2ratio, 2d_I] in/out */
+  uint16_t* idx_state_score;
+  uint16_t* cache;             /* dev, entry g at cache + b*cache_bstride + g*d */
+  int64_t cache_bstride;
+  uint16_t* idx_cache;         /* dev, entry g at idx_cache + b*idx_bstride + g*d_I */
+  int64_t idx_bstride;
+  int max_entries;
+  uint16_t* ring;              /* dev, slot j at ring + b*ring_bstride + j*d */
+  int64_t ring_bstride;
+  int ring_cap;
+  int32_t* topk_idx;           /* dev [B, topk] out: the selection used */
+  float* cache_f32;            /* nullable dev, as cache: the new main entry before rounding */
+  void* out;                   /* dev [B, H, d] */
+  int out_is_f32;
+  void* ws;
+  size_t ws_bytes;             /* >= csa_workspace_size(CSA_WS_DECODE_FUSED, B, 1, max_entries, topk) */
+  void* const* stage_events;   /* nullable: 5 cudaEvent_t recorded on the stream before the compressor
+                                  step, after it, after the indexer, after top-k and after attention */
+} csa_decode_args;
+
+/*
+ * csa_decode_fused -- one CSA decode step ([P5] §2 order): the C4A step of the main and index
+ * streams (writing entry pos//ratio of both caches when (pos+1)%ratio == 0, then rolling the
+ * state), the window-ring write of slot pos % ring_cap, the indexer over the (pos+1)//ratio
+ * visible entries, top-k, sparse MQA with the sink and inverse RoPE. Stream-ordered; no host
+ * synchronisation, so it can be captured in a CUDA graph.
+ */
+CSA_API int csa_decode_fused(const csa_decode_args* a, void* stream);
+
+/* Arguments of one HCA decode step (C128A, no index module). */
+typedef struct {
+  int B;
+  int H, d, rope_dim;          /* 128, 512, 64 */
+  int ratio;                   /* 128 */
+  int window;                  /* 128 */
+  float rope_base, eps, scale;
+  const int32_t* pos;          /* dev [B] */
+  const uint16_t* kv;          /* dev [B, d] */
+  const uint16_t* score;       /* dev [B, d] */
+  const uint16_t* win_kv;      /* dev [B, d] */
+  const uint16_t* q;           /* dev [B, H, d] */
+  const float* sink;           /* dev [H] */
+  const uint16_t* gamma;       /* dev [d] */
+  uint16_t* state_kv;          /* dev [B, ratio, d] in/out */
+  uint16_t* state_score;
+  uint16_t* cache;
+  int64_t cache_bstride;
+  int max_entries;
+  uint16_t* ring;
+  int64_t ring_bstride;
+  int ring_cap;
+  float* cache_f32;            /* nullable */
+  void* out;
+  int out_is_f32;
+  void* ws;
+  size_t ws_bytes;
+  void* const* stage_events;   /* nullable: 3 cudaEvent_t recorded before the C128A step, after it and
+                                  after attention */
+} hca_decode_args;
+
+/* hca_decode_fused -- one HCA decode step ([P5] §3): C128A step, window write, hca_attn. */
+CSA_API int hca_decode_fused(const hca_decode_args* a, void* stream);
+
+/*
+ * csa_get_device_status -- synchronise `stream`, read the status word in `ws` into *status
+ * (CSA_OK, CSA_ERR_TIMEOUT or CSA_ERR_BOUNDS) and clear it. Returns CSA_ERR_CUDA if the
+ * stream itself reports an error.
+ */
+CSA_API int csa_get_device_status(void* ws, void* stream, int* status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_H_ */

@@ -1,0 +1,607 @@
+// api.cu -- the C ABI of libcsa.so (declared in include/csa.h): argument checks, workspace
+// layout, TMA descriptor encoding and the launch sequence of every entry point.
+//
+// The library never allocates device memory. Scratch space (the indexer's score rows and the
+// top-k merge lists) lives in the caller's workspace; its first 256 bytes are the device
+// status word that kernels set instead of trapping.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "csa.h"
+#include "kernels.cuh"
+
+namespace csa {
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define CSA_CHECK_ARG(cond, ...)                                   \
+  do {                                                             \
+    if (!(cond)) return fail(CSA_ERR_INVALID_ARG, __VA_ARGS__);    \
+  } while (0)
+#define CSA_CHECK_SUP(cond, ...)                                   \
+  do {                                                             \
+    if (!(cond)) return fail(CSA_ERR_UNSUPPORTED, __VA_ARGS__);    \
+  } while (0)
+#define CSA_CUDA(call)                                                                     \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess) return fail(CSA_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- TMA descriptors through the runtime's driver entry point (no link-time libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encoder(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (fn == nullptr) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *out = fn;
+  return CSA_OK;
+}
+
+// 2D bf16 tensor [rows, cols] with row pitch `pitch_elems`, box {box_cols, box_rows}, 128B swizzle.
+int make_map_2d(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows, uint64_t pitch_elems,
+                uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc;
+  if (int rc = get_encoder(&enc)) return rc;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {pitch_elems * 2};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return CSA_OK;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem = 0;
+  bool attrs_set = false;
+};
+
+int device_info(DeviceInfo** out) {
+  static DeviceInfo info[64];
+  static std::mutex mu;
+  int dev = 0;
+  CSA_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(CSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  DeviceInfo& d = info[dev];
+  if (!d.attrs_set) {
+    CSA_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    CSA_CUDA(cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    int cc_major = 0, cc_minor = 0;
+    CSA_CUDA(cudaDeviceGetAttribute(&cc_major, cudaDevAttrComputeCapabilityMajor, dev));
+    CSA_CUDA(cudaDeviceGetAttribute(&cc_minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (cc_major != 10 || cc_minor != 0)
+      return fail(CSA_ERR_UNSUPPORTED, "libcsa is built for sm_100a; device is sm_%d%d", cc_major, cc_minor);
+    const int ms = d.max_smem;
+    CSA_CUDA(cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTopkChunk * 4));
+    d.attrs_set = true;
+  }
+  *out = &d;
+  return CSA_OK;
+}
+
+// ---- workspace layout
+struct IdxWs {
+  size_t scores_off, cand_key_off, cand_idx_off, cand_cnt_off, total;
+  int max_chunks;
+};
+
+IdxWs indexer_ws_layout(long long queries, int max_entries, int topk) {
+  IdxWs w{};
+  size_t off = kStatusBytes;
+  w.scores_off = off;
+  off = round_up(off + (size_t)queries * (size_t)max_entries * 4, 256);
+  w.max_chunks = max_entries > kTopkChunk ? (max_entries + kTopkChunk - 1) / kTopkChunk : 0;
+  w.cand_key_off = off;
+  off = round_up(off + (size_t)queries * w.max_chunks * topk * 4, 256);
+  w.cand_idx_off = off;
+  off = round_up(off + (size_t)queries * w.max_chunks * topk * 4, 256);
+  w.cand_cnt_off = off;
+  off = round_up(off + (size_t)queries * w.max_chunks * 4, 256);
+  w.total = off;
+  return w;
+}
+
+int check_ws(const void* ws, size_t ws_bytes, size_t need) {
+  if (ws == nullptr || !aligned(ws, 256)) return fail(CSA_ERR_WORKSPACE, "workspace null or not 256-byte aligned");
+  if (ws_bytes < need) return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", ws_bytes, need);
+  return CSA_OK;
+}
+
+int check_cfg(const csa_compressor_cfg* c) {
+  CSA_CHECK_ARG(c != nullptr, "cfg is null");
+  CSA_CHECK_SUP((c->ratio == 4 && c->overlap == 1) || (c->ratio == 128 && c->overlap == 0),
+                "(ratio, overlap) must be (4,1) or (128,0)");
+  CSA_CHECK_SUP(c->d == 128 || c->d == 512, "d must be 128 or 512");
+  CSA_CHECK_SUP(c->rope_dim >= 8 && c->rope_dim % 8 == 0 && c->rope_dim <= c->d && c->rope_dim / 2 <= kMaxRopePairs,
+                "rope_dim must be a multiple of 8 in [8, min(d, 128)]");
+  CSA_CHECK_ARG(std::isfinite(c->rope_base) && c->rope_base > 0.f, "rope_base must be positive");
+  CSA_CHECK_ARG(std::isfinite(c->eps) && c->eps >= 0.f, "eps must be >= 0");
+  return CSA_OK;
+}
+
+CompressParams compress_params(const csa_compressor_cfg* c, int B, int S, const int32_t* start_pos, const uint16_t* kv,
+                               const uint16_t* score, const uint16_t* gamma, uint16_t* skv, uint16_t* ssc,
+                               uint16_t* cache, int64_t cache_bstride, int max_entries, float* cache_f32,
+                               uint32_t* status) {
+  CompressParams p{};
+  p.ratio = c->ratio;
+  p.overlap = c->overlap;
+  p.d = c->d;
+  p.rope_dim = c->rope_dim;
+  p.rope_base = c->rope_base;
+  p.eps = c->eps;
+  p.B = B;
+  p.S = S;
+  p.start_pos = start_pos;
+  p.kv = kv;
+  p.score = score;
+  p.gamma = gamma;
+  p.state_kv = skv;
+  p.state_score = ssc;
+  p.cache = cache;
+  p.cache_bstride = cache_bstride;
+  p.max_entries = max_entries;
+  p.cache_f32 = cache_f32;
+  p.fuse_state = S == 1 ? 1 : 0;
+  p.status = status;
+  return p;
+}
+
+int check_compress_args(const csa_compressor_cfg* cfg, int B, int S, const int32_t* start_pos, const uint16_t* kv,
+                        const uint16_t* score, const uint16_t* gamma, const uint16_t* skv, const uint16_t* ssc,
+                        const uint16_t* cache, int64_t cache_bstride, int max_entries, const float* cache_f32) {
+  if (int rc = check_cfg(cfg)) return rc;
+  CSA_CHECK_ARG(B > 0 && S > 0, "B and S must be positive");
+  CSA_CHECK_ARG(start_pos && kv && score && gamma && skv && ssc && cache, "null pointer argument");
+  CSA_CHECK_ARG(aligned(kv, 16) && aligned(score, 16) && aligned(gamma, 16) && aligned(skv, 16) &&
+                    aligned(ssc, 16) && aligned(cache, 16) && aligned(start_pos, 4),
+                "pointers must be 16-byte aligned");
+  CSA_CHECK_ARG(cache_f32 == nullptr || aligned(cache_f32, 16), "cache_f32 must be 16-byte aligned");
+  CSA_CHECK_ARG(max_entries > 0, "max_entries must be positive");
+  CSA_CHECK_ARG(cache_bstride >= (int64_t)max_entries * cfg->d && cache_bstride % 8 == 0,
+                "cache_bstride must be >= max_entries*d and a multiple of 8");
+  return CSA_OK;
+}
+
+int launch_compress(const CompressLaunch& L, int nstreams, int B, int S, int ratio, cudaStream_t st) {
+  const dim3 grid((unsigned)((S + ratio - 1) / ratio), (unsigned)B, (unsigned)nstreams);
+  compress_kernel<<<grid, kCompressThreads, 0, st>>>(L);
+  CSA_CUDA(cudaGetLastError());
+  if (S > 1) {
+    compress_state_kernel<<<dim3((unsigned)B, 1, (unsigned)nstreams), kCompressThreads, 0, st>>>(L);
+    CSA_CUDA(cudaGetLastError());
+  }
+  return CSA_OK;
+}
+
+// ---- indexer + top-k
+struct IndexerArgs {
+  int B, S, H_I, d_I, ratio, topk;
+  const int32_t* q_pos;
+  const uint16_t* q_idx;
+  const float* w;
+  const uint16_t* idx_cache;
+  int64_t idx_bstride;
+  int max_entries;
+  int32_t* topk_idx;
+  float* scores_opt;
+  void* ws;
+  size_t ws_bytes;
+};
+
+int check_indexer_args(const IndexerArgs& a) {
+  CSA_CHECK_ARG(a.B > 0 && a.S > 0, "B and S must be positive");
+  CSA_CHECK_SUP(a.d_I == 128, "d_I must be 128");
+  CSA_CHECK_SUP(a.H_I == 4 || a.H_I == 8 || a.H_I == 16 || a.H_I == 32 || a.H_I == 64 || a.H_I == 128,
+                "H_I must be a power of two in [4, 128]");
+  CSA_CHECK_ARG(a.ratio > 0, "ratio must be positive");
+  CSA_CHECK_SUP(a.topk >= 1 && a.topk <= kAttnMaxTopk, "topk must be in [1, %d]", kAttnMaxTopk);
+  CSA_CHECK_SUP(a.max_entries >= 1 && a.max_entries <= (1 << 24), "max_entries must be in [1, 2^24]");
+  CSA_CHECK_ARG(a.q_pos && a.q_idx && a.w && a.idx_cache && a.topk_idx, "null pointer argument");
+  CSA_CHECK_ARG(aligned(a.q_idx, 16) && aligned(a.idx_cache, 16) && aligned(a.w, 4) && aligned(a.topk_idx, 4) &&
+                    aligned(a.q_pos, 4),
+                "misaligned pointer");
+  CSA_CHECK_ARG(a.idx_bstride >= (int64_t)a.max_entries * a.d_I && a.idx_bstride % a.d_I == 0,
+                "idx_bstride must be >= max_entries*d_I and a multiple of d_I");
+  CSA_CHECK_ARG(a.scores_opt == nullptr || aligned(a.scores_opt, 4), "scores_opt misaligned");
+  const long long rows = (long long)a.B * (a.idx_bstride / a.d_I);
+  CSA_CHECK_SUP(rows < (1ll << 31), "index cache too large for 32-bit row coordinates");
+  const long long qrows = (long long)a.B * a.S * a.H_I;
+  CSA_CHECK_SUP(qrows < (1ll << 31), "too many query rows");
+  return CSA_OK;
+}
+
+int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* ev = nullptr) {
+  DeviceInfo* dev;
+  if (int rc = device_info(&dev)) return rc;
+  const long long queries = (long long)a.B * a.S;
+  const IdxWs L = indexer_ws_layout(queries, a.max_entries, a.topk);
+  if (int rc = check_ws(a.ws, a.ws_bytes, L.total)) return rc;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  float* scores = a.scores_opt ? a.scores_opt : reinterpret_cast<float*>(ws + L.scores_off);
+
+  IndexerParams P{};
+  P.B = a.B;
+  P.S = a.S;
+  P.QG = a.S == 1 ? 1 : std::min(a.S, 256 / a.H_I);
+  P.N = (int)round_up((size_t)P.QG * a.H_I, 16);
+  P.ratio = a.ratio;
+  P.max_entries = a.max_entries;
+  P.groups_per_req = (a.S + P.QG - 1) / P.QG;
+  P.tiles_per_group = (a.max_entries + 127) / 128;
+  P.total_items = (long long)a.B * P.groups_per_req * P.tiles_per_group;
+  P.rows_per_req = a.idx_bstride / a.d_I;
+  int stages = kIdxMaxStages;
+  while (stages > 2 && indexer_smem_bytes(stages, P.N) > (size_t)dev->max_smem) --stages;
+  CSA_CHECK_SUP(indexer_smem_bytes(stages, P.N) <= (size_t)dev->max_smem, "shared memory too small for the indexer");
+  P.stages = stages;
+  int cols = 32;
+  while (cols < 2 * P.N) cols <<= 1;
+  P.tmem_cols = cols;
+  P.q_pos = a.q_pos;
+  P.w = a.w;
+  P.scores = scores;
+  P.scores_stride = a.max_entries;
+  P.status = status;
+
+  CUtensorMap map_k, map_q;
+  if (int rc = make_map_2d(&map_k, a.idx_cache, 128, (uint64_t)a.B * P.rows_per_req, 128, 64, 128)) return rc;
+  if (int rc = make_map_2d(&map_q, a.q_idx, 128, (uint64_t)queries * a.H_I, 128, 64, (uint32_t)P.N)) return rc;
+  const size_t smem = indexer_smem_bytes(stages, P.N);
+  const unsigned grid = (unsigned)std::min<long long>(P.total_items, dev->sms);
+  switch (a.H_I) {
+    case 4: indexer_kernel<4><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
+    case 8: indexer_kernel<8><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
+    case 16: indexer_kernel<16><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
+    case 32: indexer_kernel<32><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
+    case 64: indexer_kernel<64><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
+    default: indexer_kernel<128><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
+  }
+  CSA_CUDA(cudaGetLastError());
+  if (ev) CSA_CUDA(cudaEventRecord(ev[0], st));
+
+  TopkParams T{};
+  T.topk = a.topk;
+  T.ratio = a.ratio;
+  T.max_entries = a.max_entries;
+  T.chunk = kTopkChunk;
+  T.max_chunks = L.max_chunks;
+  T.q_pos = a.q_pos;
+  T.scores = scores;
+  T.scores_stride = a.max_entries;
+  T.out = a.topk_idx;
+  T.cand_key = reinterpret_cast<uint32_t*>(ws + L.cand_key_off);
+  T.cand_idx = reinterpret_cast<int32_t*>(ws + L.cand_idx_off);
+  T.cand_cnt = reinterpret_cast<int*>(ws + L.cand_cnt_off);
+  T.status = status;
+  const int nchunks = std::max(1, L.max_chunks);
+  const size_t tsmem = (size_t)std::min(a.max_entries, kTopkChunk) * 4;
+  topk_chunk_kernel<<<dim3((unsigned)nchunks, (unsigned)queries), kTopkThreads, tsmem, st>>>(T);
+  CSA_CUDA(cudaGetLastError());
+  if (L.max_chunks > 1) {
+    CSA_CHECK_SUP(L.max_chunks <= kTopkMaxChunks, "max_entries too large for the top-k merge");
+    topk_merge_kernel<<<(unsigned)queries, kTopkThreads, 0, st>>>(T);
+    CSA_CUDA(cudaGetLastError());
+  }
+  if (ev) CSA_CUDA(cudaEventRecord(ev[1], st));
+  return CSA_OK;
+}
+
+// ---- attention
+struct AttnArgs {
+  int B, S, H, d, rope_dim;
+  float rope_base, scale;
+  int ratio;
+  const int32_t* q_pos;
+  const uint16_t* q;
+  const uint16_t* ring;
+  int64_t ring_bstride;
+  int ring_cap, window;
+  const uint16_t* cache;
+  int64_t cache_bstride;
+  int max_entries;
+  const int32_t* topk_idx;
+  int topk;
+  const float* sink;
+  void* out;
+  int out_is_f32;
+  void* ws;
+  size_t ws_bytes;
+};
+
+int check_attn_args(const AttnArgs& a, bool csa_mode) {
+  CSA_CHECK_ARG(a.B > 0 && a.S > 0, "B and S must be positive");
+  CSA_CHECK_SUP(a.d == 512, "d must be 512");
+  CSA_CHECK_SUP(a.H >= 1 && a.H <= 128, "H must be in [1, 128]");
+  CSA_CHECK_SUP(a.rope_dim >= 2 && a.rope_dim % 2 == 0 && a.rope_dim <= 256 && a.rope_dim / 2 <= kMaxRopePairs,
+                "rope_dim must be even and <= 128");
+  CSA_CHECK_ARG(std::isfinite(a.rope_base) && a.rope_base > 0.f, "rope_base must be positive");
+  CSA_CHECK_ARG(std::isfinite(a.scale), "scale must be finite");
+  CSA_CHECK_ARG(a.ratio > 0, "ratio must be positive");
+  CSA_CHECK_SUP(a.window >= 1 && a.window <= kAttnMaxWindow, "window must be in [1, %d]", kAttnMaxWindow);
+  CSA_CHECK_ARG(a.ring_cap >= a.window, "ring_cap must be >= window");
+  CSA_CHECK_ARG(a.max_entries >= 1, "max_entries must be positive");
+  CSA_CHECK_ARG(a.q_pos && a.q && a.ring && a.cache && a.sink && a.out, "null pointer argument");
+  CSA_CHECK_ARG(aligned(a.q, 16) && aligned(a.ring, 16) && aligned(a.cache, 16) && aligned(a.out, 16) &&
+                    aligned(a.sink, 4) && aligned(a.q_pos, 4),
+                "misaligned pointer");
+  CSA_CHECK_ARG(a.ring_bstride % a.d == 0 && a.ring_bstride >= (int64_t)a.ring_cap * a.d,
+                "ring_bstride must be a multiple of d and >= ring_cap*d");
+  CSA_CHECK_ARG(a.cache_bstride % a.d == 0 && a.cache_bstride >= (int64_t)a.max_entries * a.d,
+                "cache_bstride must be a multiple of d and >= max_entries*d");
+  CSA_CHECK_SUP((long long)a.B * (a.ring_bstride / a.d) < (1ll << 30) &&
+                    (long long)a.B * (a.cache_bstride / a.d) < (1ll << 30),
+                "ring or cache too large for 30-bit row coordinates");
+  CSA_CHECK_SUP((long long)a.B * a.S * a.H < (1ll << 31), "too many query rows");
+  if (csa_mode) {
+    CSA_CHECK_ARG(a.topk_idx != nullptr && aligned(a.topk_idx, 4), "topk_idx null or misaligned");
+    CSA_CHECK_SUP(a.topk >= 1 && a.topk <= kAttnMaxTopk, "topk must be in [1, %d]", kAttnMaxTopk);
+  }
+  return check_ws(a.ws, a.ws_bytes, kStatusBytes);
+}
+
+int run_attn(const AttnArgs& a, bool csa_mode, cudaStream_t st) {
+  DeviceInfo* dev;
+  if (int rc = device_info(&dev)) return rc;
+  AttnParams P{};
+  P.B = a.B;
+  P.S = a.S;
+  P.H = a.H;
+  P.d = a.d;
+  P.rope_dim = a.rope_dim;
+  P.rope_base = a.rope_base;
+  P.scale_log2 = a.scale * 1.4426950408889634f;
+  P.window = a.window;
+  P.ring_cap = a.ring_cap;
+  P.ring_rows = a.ring_bstride / a.d;
+  P.cache_rows = a.cache_bstride / a.d;
+  P.max_entries = a.max_entries;
+  P.ratio = a.ratio;
+  P.q_pos = a.q_pos;
+  P.topk_idx = csa_mode ? a.topk_idx : nullptr;
+  P.topk = csa_mode ? a.topk : 0;
+  P.sink = a.sink;
+  P.out = a.out;
+  P.out_is_f32 = a.out_is_f32 ? 1 : 0;
+  P.status = reinterpret_cast<uint32_t*>(a.ws);
+  P.ring = a.ring;
+  P.cache = a.cache;
+  CUtensorMap map_q;
+  const long long queries = (long long)a.B * a.S;
+  if (int rc = make_map_2d(&map_q, a.q, 512, (uint64_t)queries * a.H, 512, 64, 128)) return rc;
+  const size_t smem = attn_smem_bytes();
+  CSA_CHECK_SUP(smem <= (size_t)dev->max_smem, "shared memory too small for the attention kernel");
+  CSA_CHECK_SUP(queries <= 65535, "at most 65535 queries per call");
+  attn_kernel<<<dim3(2, (unsigned)queries), kAttnThreads, smem, st>>>(map_q, P);
+  CSA_CUDA(cudaGetLastError());
+  return CSA_OK;
+}
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+const char* csa_status_string(int status) {
+  switch (status) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_INVALID_ARG: return "invalid argument";
+    case CSA_ERR_UNSUPPORTED: return "unsupported shape";
+    case CSA_ERR_CUDA: return "CUDA error";
+    case CSA_ERR_TIMEOUT: return "device wait timed out";
+    case CSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case CSA_ERR_BOUNDS: return "index out of range";
+    default: return "unknown status";
+  }
+}
+
+const char* csa_last_error(void) { return g_err; }
+
+int csa_version(void) { return 1; }
+
+int csa_workspace_size(int kind, int B, int S, int max_entries, int topk, size_t* bytes) {
+  CSA_CHECK_ARG(bytes != nullptr, "bytes is null");
+  CSA_CHECK_ARG(B > 0 && S > 0 && max_entries > 0, "B, S and max_entries must be positive");
+  switch (kind) {
+    case CSA_WS_INDEXER_TOPK:
+    case CSA_WS_DECODE_FUSED:
+      CSA_CHECK_ARG(topk > 0, "topk must be positive");
+      *bytes = indexer_ws_layout((long long)B * S, max_entries, topk).total;
+      return CSA_OK;
+    case CSA_WS_SPARSE_ATTN:
+    case CSA_WS_HCA_ATTN:
+    case CSA_WS_HCA_DECODE_FUSED:
+      *bytes = kStatusBytes;
+      return CSA_OK;
+    default:
+      return fail(CSA_ERR_INVALID_ARG, "unknown workspace kind %d", kind);
+  }
+}
+
+int csa_state_reset(const csa_compressor_cfg* cfg, int B, uint16_t* state_kv, uint16_t* state_score, void* stream) {
+  if (int rc = check_cfg(cfg)) return rc;
+  CSA_CHECK_ARG(B > 0 && state_kv && state_score, "bad arguments");
+  const long long n = (long long)B * (1 + cfg->overlap) * cfg->ratio * (1 + cfg->overlap) * cfg->d;
+  const int blocks = (int)std::min<long long>((n + 255) / 256, 4096);
+  state_reset_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(state_kv, state_score, n);
+  CSA_CUDA(cudaGetLastError());
+  return CSA_OK;
+}
+
+int csa_compress(const csa_compressor_cfg* cfg, int B, int S, const int32_t* start_pos, const uint16_t* kv,
+                 const uint16_t* score, const uint16_t* gamma, uint16_t* state_kv, uint16_t* state_score,
+                 uint16_t* cache, int64_t cache_bstride, int max_entries, float* cache_f32, void* stream) {
+  if (int rc = check_compress_args(cfg, B, S, start_pos, kv, score, gamma, state_kv, state_score, cache,
+                                   cache_bstride, max_entries, cache_f32))
+    return rc;
+  CompressLaunch L{};
+  L.p[0] = compress_params(cfg, B, S, start_pos, kv, score, gamma, state_kv, state_score, cache, cache_bstride,
+                           max_entries, cache_f32, nullptr);
+  L.p[1] = L.p[0];
+  return launch_compress(L, 1, B, S, cfg->ratio, static_cast<cudaStream_t>(stream));
+}
+
+int csa_indexer_topk(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
+                     const uint16_t* q_idx, const float* w, const uint16_t* idx_cache, int64_t idx_bstride,
+                     int max_entries, int32_t* topk_idx, float* scores_opt, void* ws, size_t ws_bytes,
+                     void* stream) {
+  IndexerArgs a{B, S, H_I, d_I, ratio, topk, q_pos, q_idx, w, idx_cache, idx_bstride, max_entries, topk_idx,
+                scores_opt, ws, ws_bytes};
+  if (int rc = check_indexer_args(a)) return rc;
+  return run_indexer_topk(a, static_cast<cudaStream_t>(stream));
+}
+
+int csa_sparse_attn(int B, int S, int H, int d, int rope_dim, float rope_base, float scale, const int32_t* q_pos,
+                    const uint16_t* q, const uint16_t* ring, int64_t ring_bstride, int ring_cap, int window,
+                    const uint16_t* cache, int64_t cache_bstride, int max_entries, const int32_t* topk_idx, int topk,
+                    const float* sink, void* out, int out_is_f32, void* ws, size_t ws_bytes, void* stream) {
+  AttnArgs a{B, S, H, d, rope_dim, rope_base, scale, 4, q_pos, q, ring, ring_bstride, ring_cap, window, cache,
+             cache_bstride, max_entries, topk_idx, topk, sink, out, out_is_f32, ws, ws_bytes};
+  if (int rc = check_attn_args(a, true)) return rc;
+  return run_attn(a, true, static_cast<cudaStream_t>(stream));
+}
+
+int hca_attn(int B, int S, int H, int d, int rope_dim, float rope_base, float scale, int ratio, const int32_t* q_pos,
+             const uint16_t* q, const uint16_t* ring, int64_t ring_bstride, int ring_cap, int window,
+             const uint16_t* cache, int64_t cache_bstride, int max_entries, const float* sink, void* out,
+             int out_is_f32, void* ws, size_t ws_bytes, void* stream) {
+  AttnArgs a{B, S, H, d, rope_dim, rope_base, scale, ratio, q_pos, q, ring, ring_bstride, ring_cap, window, cache,
+             cache_bstride, max_entries, nullptr, 0, sink, out, out_is_f32, ws, ws_bytes};
+  if (int rc = check_attn_args(a, false)) return rc;
+  return run_attn(a, false, static_cast<cudaStream_t>(stream));
+}
+
+int csa_decode_fused(const csa_decode_args* a, void* stream) {
+  CSA_CHECK_ARG(a != nullptr, "args is null");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const csa_compressor_cfg main_cfg{a->ratio, 1, a->d, a->rope_dim, a->rope_base, a->eps};
+  const csa_compressor_cfg idx_cfg{a->ratio, 1, a->d_I, a->rope_dim, a->rope_base, a->eps};
+  CSA_CHECK_SUP(a->ratio == 4, "CSA decode uses ratio 4");
+  if (int rc = check_compress_args(&main_cfg, a->B, 1, a->pos, a->kv, a->score, a->gamma, a->state_kv,
+                                   a->state_score, a->cache, a->cache_bstride, a->max_entries, a->cache_f32))
+    return rc;
+  if (int rc = check_compress_args(&idx_cfg, a->B, 1, a->pos, a->idx_kv, a->idx_score, a->idx_gamma,
+                                   a->idx_state_kv, a->idx_state_score, a->idx_cache, a->idx_bstride,
+                                   a->max_entries, nullptr))
+    return rc;
+  CSA_CHECK_ARG(a->win_kv && aligned(a->win_kv, 16), "win_kv null or misaligned");
+  IndexerArgs ia{a->B, 1, a->H_I, a->d_I, a->ratio, a->topk, a->pos, a->q_idx, a->w, a->idx_cache, a->idx_bstride,
+                 a->max_entries, a->topk_idx, nullptr, a->ws, a->ws_bytes};
+  if (int rc = check_indexer_args(ia)) return rc;
+  AttnArgs aa{a->B, 1, a->H, a->d, a->rope_dim, a->rope_base, a->scale, a->ratio, a->pos, a->q, a->ring,
+              a->ring_bstride, a->ring_cap, a->window, a->cache, a->cache_bstride, a->max_entries, a->topk_idx,
+              a->topk, a->sink, a->out, a->out_is_f32, a->ws, a->ws_bytes};
+  if (int rc = check_attn_args(aa, true)) return rc;
+  const IdxWs L = indexer_ws_layout(a->B, a->max_entries, a->topk);
+  if (int rc = check_ws(a->ws, a->ws_bytes, L.total)) return rc;
+
+  uint32_t* status = static_cast<uint32_t*>(a->ws);
+  CompressLaunch CL{};
+  CL.p[0] = compress_params(&main_cfg, a->B, 1, a->pos, a->kv, a->score, a->gamma, a->state_kv, a->state_score,
+                            a->cache, a->cache_bstride, a->max_entries, a->cache_f32, status);
+  CL.p[0].win_src = a->win_kv;
+  CL.p[0].ring = a->ring;
+  CL.p[0].ring_bstride = a->ring_bstride;
+  CL.p[0].ring_cap = a->ring_cap;
+  CL.p[1] = compress_params(&idx_cfg, a->B, 1, a->pos, a->idx_kv, a->idx_score, a->idx_gamma, a->idx_state_kv,
+                            a->idx_state_score, a->idx_cache, a->idx_bstride, a->max_entries, nullptr, status);
+  cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(a->stage_events);
+  if (ev) CSA_CUDA(cudaEventRecord(ev[0], st));
+  if (int rc = launch_compress(CL, 2, a->B, 1, a->ratio, st)) return rc;
+  if (ev) CSA_CUDA(cudaEventRecord(ev[1], st));
+  if (int rc = run_indexer_topk(ia, st, ev ? ev + 2 : nullptr)) return rc;
+  if (int rc = run_attn(aa, true, st)) return rc;
+  if (ev) CSA_CUDA(cudaEventRecord(ev[4], st));
+  return CSA_OK;
+}
+
+int hca_decode_fused(const hca_decode_args* a, void* stream) {
+  CSA_CHECK_ARG(a != nullptr, "args is null");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const csa_compressor_cfg cfg{a->ratio, 0, a->d, a->rope_dim, a->rope_base, a->eps};
+  CSA_CHECK_SUP(a->ratio == 128, "HCA decode uses ratio 128");
+  if (int rc = check_compress_args(&cfg, a->B, 1, a->pos, a->kv, a->score, a->gamma, a->state_kv, a->state_score,
+                                   a->cache, a->cache_bstride, a->max_entries, a->cache_f32))
+    return rc;
+  CSA_CHECK_ARG(a->win_kv && aligned(a->win_kv, 16), "win_kv null or misaligned");
+  AttnArgs aa{a->B, 1, a->H, a->d, a->rope_dim, a->rope_base, a->scale, a->ratio, a->pos, a->q, a->ring,
+              a->ring_bstride, a->ring_cap, a->window, a->cache, a->cache_bstride, a->max_entries, nullptr, 0,
+              a->sink, a->out, a->out_is_f32, a->ws, a->ws_bytes};
+  if (int rc = check_attn_args(aa, false)) return rc;
+  uint32_t* status = static_cast<uint32_t*>(a->ws);
+  CompressLaunch CL{};
+  CL.p[0] = compress_params(&cfg, a->B, 1, a->pos, a->kv, a->score, a->gamma, a->state_kv, a->state_score, a->cache,
+                            a->cache_bstride, a->max_entries, a->cache_f32, status);
+  CL.p[0].win_src = a->win_kv;
+  CL.p[0].ring = a->ring;
+  CL.p[0].ring_bstride = a->ring_bstride;
+  CL.p[0].ring_cap = a->ring_cap;
+  CL.p[1] = CL.p[0];
+  cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(a->stage_events);
+  if (ev) CSA_CUDA(cudaEventRecord(ev[0], st));
+  if (int rc = launch_compress(CL, 1, a->B, 1, a->ratio, st)) return rc;
+  if (ev) CSA_CUDA(cudaEventRecord(ev[1], st));
+  if (int rc = run_attn(aa, false, st)) return rc;
+  if (ev) CSA_CUDA(cudaEventRecord(ev[2], st));
+  return CSA_OK;
+}
+
+int csa_get_device_status(void* ws, void* stream, int* status) {
+  CSA_CHECK_ARG(ws != nullptr && status != nullptr && aligned(ws, 256), "bad arguments");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  CSA_CUDA(cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st));
+  CSA_CUDA(cudaStreamSynchronize(st));
+  const uint32_t zero = 0;
+  CSA_CUDA(cudaMemcpyAsync(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice, st));
+  CSA_CUDA(cudaStreamSynchronize(st));
+  *status = (int)v;
+  return CSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,312 @@
+// compress.cu -- the C4A / C128A token compressor (K1).
+//
+// "DeepSeek-V4-Pro 架构：一个 token 的旅程", sections "压缩是逐通道的 learned pooling" and
+// "压缩条目必须等整组完成后才可见"; "图解DeepSeek V4：详细计算流程解析" §2.1 (C4A rolling state) and
+// §3.1 (C128A).
+//
+// Entry g pools, per channel c, a softmax over slots of the score stream times the kv stream:
+//   C4A  (ratio 4, overlap): 8 slots = channels [:d] of tokens 4(g-1)..4g-1 and channels [d:] of
+//        tokens 4g..4g+3; the previous-group slots of g = 0 are missing (weight 0).
+//   C128A (ratio 128): the 128 tokens of group g, one width-d stream.
+// then RMSNorm over the d channels and RoPE on the last rope_dim channels at position g*ratio.
+//
+// Work split: one CTA per (request, completed group). Each thread owns 8 consecutive channels
+// and reads them with 16-byte loads; each token's row is read once in total (the previous and
+// current halves are disjoint). Memory-bound: no tensor-core work here.
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "kernels.cuh"
+
+namespace csa {
+
+namespace {
+
+struct Vec8 {
+  float v[8];
+};
+
+__device__ __forceinline__ Vec8 load8(const uint16_t* p) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  Vec8 r;
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    r.v[2 * i] = __uint_as_float(w[i] << 16);
+    r.v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+  return r;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Where token p's stream row comes from: the segment (element offset into the kv/score inputs,
+// *from_state = false), a row of the input state (offset into the state arrays, *from_state =
+// true), or nowhere (-1: a previous group before position 0).
+__device__ __forceinline__ long long token_row(const CompressParams& P, int b, long long p, long long start,
+                                               bool* from_state) {
+  *from_state = false;
+  if (p < 0) return -1;
+  const int width = (1 + P.overlap) * P.d;
+  if (p >= start) return ((long long)b * P.S + (p - start)) * width;
+  *from_state = true;
+  const long long g0 = start / P.ratio;  // group in progress at the segment start
+  const int rows = (1 + P.overlap) * P.ratio;
+  const long long st = (long long)b * rows * width;
+  if (P.overlap) {
+    if (p / P.ratio == g0) return st + (long long)(P.ratio + p % P.ratio) * width;  // cur rows
+    if (p / P.ratio == g0 - 1) return st + (long long)(p % P.ratio) * width;        // pre rows
+    return -1;
+  }
+  if (p / P.ratio == g0) return st + (long long)(p % P.ratio) * width;
+  return -1;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int nw = (blockDim.x + 31) >> 5;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int i = 0; i < nw; ++i) s += red[i];
+  return s;
+}
+
+// Update request b's state to the state after token end-1, as the token-by-token rolling state
+// leaves it. Called by one whole CTA. The only rows that feed other rows are the C4A cur rows
+// that become pre rows when a group completes; those are read into registers before any row is
+// written.
+__device__ void update_state(const CompressParams& P, int b, long long start, long long end) {
+  const int width = (1 + P.overlap) * P.d;
+  const int rows = (1 + P.overlap) * P.ratio;
+  uint16_t* skv = P.state_kv + (long long)b * rows * width;
+  uint16_t* ssc = P.state_score + (long long)b * rows * width;
+  const int cpr = width / 8;                    // 16-byte chunks per row
+  const long long g0 = start / P.ratio;
+  const long long g_end = end / P.ratio;        // groups 0..g_end-1 are complete after the segment
+  const long long last = end - 1;
+  const bool roll = P.overlap && g_end > g0;
+  // Phase A: stash pre-row values that come from the input cur rows.
+  uint4 keep_kv[kMaxKeepChunks], keep_sc[kMaxKeepChunks];
+  if (roll) {
+    int k = 0;
+    for (int idx = threadIdx.x; idx < P.ratio * cpr && k < kMaxKeepChunks; idx += blockDim.x, ++k) {
+      const int row = idx / cpr, ch = idx % cpr;
+      const long long p = (g_end - 1) * P.ratio + row;
+      if (p < start) {
+        keep_kv[k] = *reinterpret_cast<const uint4*>(skv + (long long)(P.ratio + row) * width + ch * 8);
+        keep_sc[k] = *reinterpret_cast<const uint4*>(ssc + (long long)(P.ratio + row) * width + ch * 8);
+      }
+    }
+  }
+  __syncthreads();
+  // Phase B: every row whose newest token lies in the segment is copied from the segment.
+  for (int idx = threadIdx.x; idx < rows * cpr; idx += blockDim.x) {
+    const int row = idx / cpr, ch = idx % cpr;
+    int j;
+    if (P.overlap) {
+      if (row < P.ratio) continue;  // pre rows: phase C
+      j = row - P.ratio;
+    } else {
+      j = row;
+    }
+    const long long q = last - (((last - j) % P.ratio) + P.ratio) % P.ratio;  // newest token with q%ratio == j
+    if (q < start) continue;                                                   // unchanged
+    const long long off = ((long long)b * P.S + (q - start)) * width + ch * 8;
+    *reinterpret_cast<uint4*>(skv + (long long)row * width + ch * 8) = *reinterpret_cast<const uint4*>(P.kv + off);
+    *reinterpret_cast<uint4*>(ssc + (long long)row * width + ch * 8) = *reinterpret_cast<const uint4*>(P.score + off);
+  }
+  // Phase C: C4A pre rows <- the tokens of the last group completed in the segment.
+  if (roll) {
+    int k = 0;
+    for (int idx = threadIdx.x; idx < P.ratio * cpr && k < kMaxKeepChunks; idx += blockDim.x, ++k) {
+      const int row = idx / cpr, ch = idx % cpr;
+      const long long p = (g_end - 1) * P.ratio + row;
+      uint4 vk, vs;
+      if (p >= start) {
+        const long long off = ((long long)b * P.S + (p - start)) * width + ch * 8;
+        vk = *reinterpret_cast<const uint4*>(P.kv + off);
+        vs = *reinterpret_cast<const uint4*>(P.score + off);
+      } else {
+        vk = keep_kv[k];
+        vs = keep_sc[k];
+      }
+      *reinterpret_cast<uint4*>(skv + (long long)row * width + ch * 8) = vk;
+      *reinterpret_cast<uint4*>(ssc + (long long)row * width + ch * 8) = vs;
+    }
+  }
+}
+
+}  // namespace
+
+// grid: (group slots, B, streams); block: kCompressThreads.
+__global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaunch L) {
+  const CompressParams& P = L.p[blockIdx.z];
+  const int b = blockIdx.y;
+  if (b >= P.B) return;
+  __shared__ float red[kCompressThreads / 32];
+  __shared__ double rope_cs[2 * kMaxRopePairs];
+
+  const long long start = P.start_pos[b];
+  const long long end = start + P.S;
+  const long long g_first = start / P.ratio;
+  const long long g_last = end / P.ratio - 1;  // last group completed inside the segment
+  const long long g = g_first + blockIdx.x;
+  const int d = P.d;
+  const int tid = threadIdx.x;
+  const bool active = tid < d / 8;
+  const int c0 = tid * 8;
+
+  // Window-ring write of the fused decode step (main stream only).
+  if (P.win_src != nullptr && blockIdx.x == 0) {
+    const long long t = end - 1;
+    uint16_t* dst = P.ring + (long long)b * P.ring_bstride + (t % P.ring_cap) * d;
+    const uint16_t* src = P.win_src + (long long)b * d;
+    for (int c = tid * 8; c < d; c += blockDim.x * 8)
+      *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(src + c);
+  }
+
+  if (g <= g_last) {
+    if (g >= P.max_entries) {
+      if (tid == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    } else {
+      // Per-channel online softmax over the slots, in the log2 domain. Slots are processed in
+      // blocks of 8 whose 16-byte loads are all issued before any arithmetic.
+      float m[8], s[8], acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        m[i] = -CUDART_INF_F;
+        s[i] = 0.f;
+        acc[i] = 0.f;
+      }
+      const int nslots = P.overlap ? 2 * P.ratio : P.ratio;
+      if (active) {
+        for (int j0 = 0; j0 < nslots; j0 += 8) {
+          uint4 kraw[8], sraw[8];
+          bool have[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = j0 + u;
+            long long p;
+            int coff;
+            if (P.overlap) {
+              const bool prev = j < P.ratio;
+              p = prev ? (g - 1) * P.ratio + j : g * P.ratio + (j - P.ratio);
+              coff = prev ? c0 : d + c0;
+            } else {
+              p = g * P.ratio + j;
+              coff = c0;
+            }
+            bool from_state;
+            const long long off = token_row(P, b, p, start, &from_state);
+            have[u] = off >= 0;  // a missing slot has weight exactly 0 and is never read
+            if (have[u]) {
+              kraw[u] = *reinterpret_cast<const uint4*>((from_state ? P.state_kv : P.kv) + off + coff);
+              sraw[u] = *reinterpret_cast<const uint4*>((from_state ? P.state_score : P.score) + off + coff);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (!have[u]) continue;
+            const uint32_t kw[4] = {kraw[u].x, kraw[u].y, kraw[u].z, kraw[u].w};
+            const uint32_t sw[4] = {sraw[u].x, sraw[u].y, sraw[u].z, sraw[u].w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float kvv = __uint_as_float((i & 1) ? (kw[i >> 1] & 0xFFFF0000u) : (kw[i >> 1] << 16));
+              const float scv = __uint_as_float((i & 1) ? (sw[i >> 1] & 0xFFFF0000u) : (sw[i >> 1] << 16));
+              const float x = scv * 1.4426950408889634f;  // log2(e)
+              if (x > m[i]) {
+                const float a = exp2f(m[i] - x);
+                s[i] *= a;
+                acc[i] *= a;
+                m[i] = x;
+              }
+              const float e = exp2f(x - m[i]);
+              s[i] += e;
+              acc[i] += e * kvv;
+            }
+          }
+        }
+      }
+      float x[8];
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        x[i] = active ? acc[i] / s[i] : 0.f;
+        ss += x[i] * x[i];
+      }
+      const float tot = block_sum(ss, red);
+      const float r = rsqrtf(tot / (float)d + P.eps);
+      // RoPE table for position g*ratio: the angle is formed in double precision.
+      const int npairs = P.rope_dim / 2;
+      if (tid < npairs) {
+        const double theta = pow((double)P.rope_base, -2.0 * tid / (double)P.rope_dim);
+        double sn, cs;
+        sincos((double)(g * P.ratio) * theta, &sn, &cs);
+        rope_cs[2 * tid] = cs;
+        rope_cs[2 * tid + 1] = sn;
+      }
+      __syncthreads();
+      if (active) {
+        const Vec8 gm = load8(P.gamma + c0);
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = x[i] * r * gm.v[i];
+        const int rope0 = d - P.rope_dim;
+        if (c0 >= rope0) {
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            const int pi = (c0 + i - rope0) >> 1;
+            const float cs = (float)rope_cs[2 * pi], sn = (float)rope_cs[2 * pi + 1];
+            const float e = y[i], o = y[i + 1];
+            y[i] = e * cs - o * sn;
+            y[i + 1] = e * sn + o * cs;
+          }
+        }
+        uint16_t* dst = P.cache + (long long)b * P.cache_bstride + g * d + c0;
+        uint4 out;
+        out.x = pack_bf16x2(y[0], y[1]);
+        out.y = pack_bf16x2(y[2], y[3]);
+        out.z = pack_bf16x2(y[4], y[5]);
+        out.w = pack_bf16x2(y[6], y[7]);
+        *reinterpret_cast<uint4*>(dst) = out;
+        if (P.cache_f32 != nullptr) {
+          float* df = P.cache_f32 + (long long)b * P.cache_bstride + g * d + c0;
+          reinterpret_cast<float4*>(df)[0] = make_float4(y[0], y[1], y[2], y[3]);
+          reinterpret_cast<float4*>(df)[1] = make_float4(y[4], y[5], y[6], y[7]);
+        }
+      }
+    }
+  }
+
+  if (P.fuse_state && blockIdx.x == 0) {
+    __syncthreads();
+    update_state(P, b, start, end);
+  }
+}
+
+// Final state of a multi-token segment: one CTA per request, reads before writes.
+__global__ void __launch_bounds__(kCompressThreads) compress_state_kernel(CompressLaunch L) {
+  const CompressParams& P = L.p[blockIdx.z];
+  const int b = blockIdx.x;
+  if (b >= P.B) return;
+  const long long start = P.start_pos[b];
+  update_state(P, b, start, start + P.S);
+}
+
+// state <- kv rows 0, score rows -inf.
+__global__ void state_reset_kernel(uint16_t* kv, uint16_t* score, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    kv[i] = 0;
+    score[i] = 0xFF80;  // bf16 -inf
+  }
+}
+
+}  // namespace csa

@@ -1,0 +1,298 @@
+// indexer.cu -- lightning-indexer scores on the tcgen05 tensor cores (K2).
+//
+// "DeepSeek-V4-Pro 架构：一个 token 的旅程", section "少读 KV 之前，Indexer 仍要给历史打分": 64 heads of
+// 128 dims score every visible entry of one shared 128-dim compressed index cache,
+//     score(t, s) = sum_h w[t,h] * ReLU(q_idx[t,h,:] . k_idx[s,:]),   s < (t+1)//ratio,
+// with w free in sign (not a softmax). "图解DeepSeek V4：详细计算流程解析" §2.2: the index keys come from
+// the same 4:1 C4A compressor.
+//
+// Contraction: per work item, D[128 entries x N] = K_tile[128 x 128] . Q_group^T, where the N
+// columns are (query, head) pairs of QG consecutive queries of one request (N = QG*H_I <= 256;
+// decode: QG = 1, N = 64). A = index-cache tile (K-major, TMA, 128B swizzle), B = the group's
+// q_idx rows (K-major, TMA), D in TMEM (fp32, double-buffered). The epilogue (thread = entry =
+// TMEM lane) applies ReLU, weights by w and sums over heads, and writes one fp32 score per
+// (query, entry) with coalesced stores.
+//
+// Persistent kernel, one CTA per SM, warp roles: warp 0 = TMA producer, warp 1 = MMA issuer
+// (and TMEM owner), warps 2..5 = epilogue. Work items (request, query group, 128-entry tile) are
+// split into contiguous ranges per CTA so the Q tile of a group is loaded once per CTA. Tiles
+// past the group's last visible entry are skipped by every role alike.
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace csa {
+
+namespace {
+
+struct ItemCoord {
+  int b, qg, et;
+};
+
+// Visible entries of query (b, i): (t+1)//ratio, capped at max_entries.
+__device__ __forceinline__ int visible_of(const IndexerParams& P, int b, int i) {
+  const int t = P.q_pos[(long long)b * P.S + i];
+  int E = (t + 1) / P.ratio;
+  E = E < 0 ? 0 : E;
+  return E > P.max_entries ? P.max_entries : E;
+}
+
+// Walks the work items [it, it1) that hold at least one visible entry, in order, and numbers
+// the query groups met (gi). Every role runs its own copy over the same range.
+struct ItemIter {
+  long long it, it1;
+  int cur_b, cur_qg, gv, gi;
+  bool started;
+
+  __device__ ItemIter(long long a, long long b) : it(a), it1(b), cur_b(-1), cur_qg(-1), gv(0), gi(-1), started(false) {}
+
+  __device__ bool next(const IndexerParams& P, ItemCoord& c, bool& new_group) {
+    while (it < it1) {
+      const long long x = it++;
+      c.et = (int)(x % P.tiles_per_group);
+      const long long gq = x / P.tiles_per_group;
+      c.qg = (int)(gq % P.groups_per_req);
+      c.b = (int)(gq / P.groups_per_req);
+      if (c.b != cur_b || c.qg != cur_qg) {
+        cur_b = c.b;
+        cur_qg = c.qg;
+        started = false;
+        gv = 0;
+        const int i0 = c.qg * P.QG, i1 = min(P.S, i0 + P.QG);
+        for (int i = i0; i < i1; ++i) gv = max(gv, visible_of(P, c.b, i));
+      }
+      if (c.et * 128 >= gv) continue;
+      new_group = !started;
+      if (new_group) {
+        ++gi;
+        started = true;
+      }
+      return true;
+    }
+    return false;
+  }
+};
+
+struct IdxSmem {
+  uint64_t k_full[kIdxMaxStages], k_empty[kIdxMaxStages];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  float w[256];
+  int vis[256];
+};
+
+template <int HI>
+__device__ __forceinline__ void epilogue_tile(const IndexerParams& P, const IdxSmem& sm, uint32_t tmem_acc, int b,
+                                              int qg, int et, int row) {
+  constexpr int kQPerChunk = HI >= 32 ? 1 : 32 / HI;
+  constexpr int kChunksPerQ = HI >= 32 ? HI / 32 : 1;
+  constexpr int kColsPerQ = HI >= 32 ? 32 : HI;
+  const int nq = min(P.QG, P.S - qg * P.QG);
+  const int s = et * 128 + row;
+  const int ncols = nq * HI;
+  for (int col0 = 0; col0 < ncols; col0 += 32 * kChunksPerQ) {
+    float sigma[kQPerChunk];
+#pragma unroll
+    for (int j = 0; j < kQPerChunk; ++j) sigma[j] = 0.f;
+#pragma unroll
+    for (int c = 0; c < kChunksPerQ; ++c) {
+      uint32_t v[32];
+      tmem_ld32(tmem_acc + col0 + 32 * c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float x = __uint_as_float(v[j]);
+        sigma[j / kColsPerQ] = fmaf(sm.w[col0 + 32 * c + j], fmaxf(x, 0.f), sigma[j / kColsPerQ]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kQPerChunk; ++j) {
+      const int qi = col0 / HI + j;
+      if (qi < nq && s < sm.vis[qi]) {
+        const long long qrow = (long long)b * P.S + (long long)qg * P.QG + qi;
+        P.scores[qrow * P.scores_stride + s] = sigma[j];
+      }
+    }
+  }
+}
+
+}  // namespace
+
+template <int HI>
+__global__ void __launch_bounds__(kIdxThreads, 1)
+    indexer_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                   IndexerParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int NS = P.stages;
+  const int N = P.N;
+  const uint32_t q_bytes = (uint32_t)N * 256u;   // N rows x 128 dims x 2 bytes (two 64-dim blocks)
+  uint8_t* k_tiles = base;                       // NS x 32 KB: [2 d-blocks][128 rows][128 B]
+  uint8_t* q_tiles = base + (size_t)NS * 32768;  // 2 x q_bytes: [2 d-blocks][N rows][128 B]
+  IdxSmem& sm = *reinterpret_cast<IdxSmem*>(q_tiles + 2 * (size_t)q_bytes);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+      mbar_init(&sm.acc_full[i], 1);
+      mbar_init(&sm.acc_empty[i], 128);
+    }
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_k);
+    tma_prefetch_desc(&map_q);
+  }
+  const uint32_t acc_cols = (uint32_t)P.tmem_cols;  // power of two >= 2N
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, acc_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  const long long total = P.total_items;
+  const long long per = (total + gridDim.x - 1) / gridDim.x;
+  const long long it0 = min(total, (long long)blockIdx.x * per);
+  const long long it1 = min(total, it0 + per);
+  volatile int* abort_flag = &sm.abort_flag;
+  uint32_t* status = P.status;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      ItemIter iter(it0, it1);
+      ItemCoord c;
+      bool ng;
+      long long n = 0;
+      while (iter.next(P, c, ng)) {
+        if (ng) {
+          const int slot = iter.gi & 1;
+          if (!mbar_wait(&sm.q_empty[slot], ((iter.gi >> 1) & 1) ^ 1, abort_flag, status, 201)) break;
+          mbar_arrive_expect_tx(&sm.q_full[slot], q_bytes);
+          const int row0 = (int)(((long long)c.b * P.S + (long long)c.qg * P.QG) * HI);
+          uint8_t* dst = q_tiles + (size_t)slot * q_bytes;
+          tma_load_2d(dst, &map_q, 0, row0, &sm.q_full[slot]);
+          tma_load_2d(dst + (size_t)N * 128, &map_q, 64, row0, &sm.q_full[slot]);
+        }
+        const int st = (int)(n % NS);
+        const uint32_t ph = (uint32_t)((n / NS) & 1);
+        if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort_flag, status, 202)) break;
+        mbar_arrive_expect_tx(&sm.k_full[st], 32768);
+        const int krow = (int)((long long)c.b * P.rows_per_req + (long long)c.et * 128);
+        uint8_t* dst = k_tiles + (size_t)st * 32768;
+        tma_load_2d(dst, &map_k, 0, krow, &sm.k_full[st]);
+        tma_load_2d(dst + 16384, &map_k, 64, krow, &sm.k_full[st]);
+        trace_mark(status, 0, (uint32_t)(100 + n));
+        ++n;
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, N, 0, 0);
+      ItemIter iter(it0, it1);
+      ItemCoord c;
+      bool ng;
+      long long n = 0;
+      int slot = 0;
+      while (iter.next(P, c, ng)) {
+        if (ng) {
+          if (iter.gi > 0) mma_commit(&sm.q_empty[(iter.gi - 1) & 1]);  // previous group's Q is free
+          slot = iter.gi & 1;
+          if (!mbar_wait(&sm.q_full[slot], (iter.gi >> 1) & 1, abort_flag, status, 211)) break;
+        }
+        const int st = (int)(n % NS);
+        if (!mbar_wait(&sm.k_full[st], (uint32_t)((n / NS) & 1), abort_flag, status, 212)) break;
+        const int a = (int)(n & 1);
+        if (!mbar_wait(&sm.acc_empty[a], (uint32_t)(((n >> 1) & 1) ^ 1), abort_flag, status, 213)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(a * N);
+        const uint32_t ka = smem_u32(k_tiles + (size_t)st * 32768);
+        const uint32_t qa = smem_u32(q_tiles + (size_t)slot * q_bytes);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t kb = ks >> 2, off = (ks & 3) * 32;
+          const uint64_t adesc = smem_desc_sw128(ka + kb * 16384 + off, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(qa + kb * (uint32_t)N * 128 + off, 16, 1024);
+          mma_ss(d_tmem, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(&sm.k_empty[st]);
+        mma_commit(&sm.acc_full[a]);
+        trace_mark(status, 1, (uint32_t)(100 + n));
+        ++n;
+      }
+      // Every MMA issued by this thread completes before TMEM is released.
+      mma_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, abort_flag, status, 214);
+      trace_mark(status, 1, 9);
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue (warps 2..5)
+    const int et_tid = threadIdx.x - 64;              // 0..127
+    const int quad = warp & 3;                        // TMEM lanes 32*quad .. 32*quad+31
+    const int row = quad * 32 + lane;
+    ItemIter iter(it0, it1);
+    ItemCoord c;
+    bool ng;
+    long long n = 0;
+    while (iter.next(P, c, ng)) {
+      if (ng) {
+        named_bar_sync(1, 128);
+        const int nq = min(P.QG, P.S - c.qg * P.QG);
+        const long long q0 = (long long)c.b * P.S + (long long)c.qg * P.QG;
+        for (int j = et_tid; j < nq * HI; j += 128) sm.w[j] = P.w[q0 * HI + j];
+        for (int j = et_tid; j < nq; j += 128) sm.vis[j] = visible_of(P, c.b, c.qg * P.QG + j);
+        named_bar_sync(1, 128);
+      }
+      const int a = (int)(n & 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full[a], (uint32_t)((n >> 1) & 1), abort_flag, status, 221))) break;
+      if (et_tid == 0) trace_mark(status, 2, (uint32_t)(100 + n));
+      tc_fence_after();
+      epilogue_tile<HI>(P, sm, tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * N), c.b, c.qg, c.et, row);
+      tc_fence_before();
+      mbar_arrive(&sm.acc_empty[a]);
+      ++n;
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) trace_mark(status, 3, 2);
+  if (warp == 1) tmem_dealloc(tmem, acc_cols);
+  if (threadIdx.x == 32) trace_mark(status, 3, 3);
+}
+
+size_t indexer_smem_bytes(int stages, int N) {
+  return 1024 + (size_t)stages * 32768 + 2 * (size_t)N * 256 + sizeof(IdxSmem);
+}
+
+template __global__ void indexer_kernel<4>(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
+                                           IndexerParams);
+template __global__ void indexer_kernel<8>(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
+                                           IndexerParams);
+template __global__ void indexer_kernel<16>(const __grid_constant__ CUtensorMap,
+                                            const __grid_constant__ CUtensorMap, IndexerParams);
+template __global__ void indexer_kernel<32>(const __grid_constant__ CUtensorMap,
+                                            const __grid_constant__ CUtensorMap, IndexerParams);
+template __global__ void indexer_kernel<64>(const __grid_constant__ CUtensorMap,
+                                            const __grid_constant__ CUtensorMap, IndexerParams);
+template __global__ void indexer_kernel<128>(const __grid_constant__ CUtensorMap,
+                                             const __grid_constant__ CUtensorMap, IndexerParams);
+
+}  // namespace csa

@@ -1,0 +1,131 @@
+// kernels.cuh -- parameter blocks and launch constants shared by the kernels and the C ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "status.cuh"
+
+namespace csa {
+
+// ------------------------------------------------------------------------------ compressor (K1)
+
+constexpr int kCompressThreads = 256;
+constexpr int kMaxRopePairs = 64;
+// Per-thread stash of C4A cur rows that become pre rows (update_state, phase A). The host checks
+// ratio * width / 8 <= kMaxKeepChunks * kCompressThreads.
+constexpr int kMaxKeepChunks = 4;
+
+struct CompressParams {
+  int ratio, overlap, d, rope_dim;
+  float rope_base, eps;
+  int B, S;
+  const int32_t* start_pos;   // [B]
+  const uint16_t* kv;         // [B, S, width]
+  const uint16_t* score;      // [B, S, width]
+  const uint16_t* gamma;      // [d]
+  uint16_t* state_kv;         // [B, rows, width]
+  uint16_t* state_score;
+  uint16_t* cache;            // entry g of request b at cache + b*cache_bstride + g*d
+  long long cache_bstride;
+  int max_entries;
+  float* cache_f32;           // nullable, same layout as cache
+  int fuse_state;             // S == 1: the CTA of the (only) group slot also updates the state
+  // Window-ring write of the fused decode step (nullable win_src disables it).
+  const uint16_t* win_src;    // [B, d]
+  uint16_t* ring;
+  long long ring_bstride;
+  int ring_cap;
+  uint32_t* status;
+};
+
+struct CompressLaunch {
+  CompressParams p[2];        // blockIdx.z selects the stream (main / index)
+};
+
+__global__ void compress_kernel(CompressLaunch L);
+__global__ void compress_state_kernel(CompressLaunch L);
+__global__ void state_reset_kernel(uint16_t* kv, uint16_t* score, long long n);
+
+
+// ------------------------------------------------------------------------------ indexer (K2)
+
+constexpr int kIdxThreads = 192;          // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kIdxMaxStages = 8;
+
+struct IndexerParams {
+  int B, S;
+  int QG;                                 // queries per group (N = QG*H_I columns, padded to 16)
+  int N;
+  int ratio, max_entries;
+  int groups_per_req, tiles_per_group;
+  long long total_items;                  // B * groups_per_req * tiles_per_group
+  long long rows_per_req;                 // index-cache rows per request (idx_bstride / d_I)
+  int stages, tmem_cols;
+  const int32_t* q_pos;                   // [B*S]
+  const float* w;                         // [B*S, H_I]
+  float* scores;                          // [B*S, scores_stride]
+  long long scores_stride;
+  uint32_t* status;
+};
+
+template <int HI>
+__global__ void indexer_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                               IndexerParams P);
+
+// ------------------------------------------------------------------------------ top-k (K3)
+
+constexpr int kTopkThreads = 1024;
+constexpr int kTopkChunk = 16384;         // entries per chunk (staged in 64 KB of smem)
+constexpr int kTopkMaxChunks = 1024;
+
+struct TopkParams {
+  int topk, ratio, max_entries;
+  int chunk, max_chunks;
+  const int32_t* q_pos;                   // [queries]
+  const float* scores;                    // [queries, scores_stride]
+  long long scores_stride;
+  int32_t* out;                           // [queries, topk]
+  uint32_t* cand_key;                     // [queries, max_chunks, topk]
+  int32_t* cand_idx;
+  int* cand_cnt;                          // [queries, max_chunks]
+  uint32_t* status;
+};
+
+__global__ void topk_chunk_kernel(TopkParams P);
+__global__ void topk_merge_kernel(TopkParams P);
+
+// ------------------------------------------------------------------------------ attention (K4/K5)
+
+constexpr int kAttnThreads = 288;         // warps 0..3 gathers, warp 4 MMA, warps 5..8 softmax
+constexpr int kAttnMaxWindow = 1024;
+constexpr int kAttnMaxTopk = 2048;
+constexpr int kAttnMaxCompressed = 2048;  // HCA: visible entries read per query
+constexpr int kAttnMaxCands = 3200;       // window + entries + padding
+constexpr int kAttnMaxTiles = kAttnMaxCands / 64;
+
+struct AttnParams {
+  int B, S, H, d, rope_dim;
+  float rope_base, scale_log2;            // scale * log2(e)
+  int window, ring_cap;
+  long long ring_rows;                    // ring rows per request (ring_bstride / d)
+  long long cache_rows;                   // cache rows per request (cache_bstride / d)
+  int max_entries, ratio;
+  const int32_t* q_pos;                   // [B*S]
+  const uint16_t* ring;                   // row r (of B*ring_rows) at ring + r*d
+  const uint16_t* cache;                  // row r (of B*cache_rows) at cache + r*d
+  const int32_t* topk_idx;                // [B*S, topk]; null: HCA (every visible entry)
+  int topk;
+  const float* sink;                      // [H]
+  void* out;                              // [B*S, H, d]
+  int out_is_f32;
+  uint32_t* status;
+};
+
+__global__ void attn_kernel(const __grid_constant__ CUtensorMap map_q, AttnParams P);
+
+size_t attn_smem_bytes();
+size_t indexer_smem_bytes(int stages, int N);
+
+}  // namespace csa

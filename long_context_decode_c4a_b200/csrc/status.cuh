@@ -1,0 +1,70 @@
+// status.cuh -- device status word and shared constants.
+#pragma once
+
+#include <cstdint>
+
+namespace csa {
+
+// Device-side status codes (match csa_status in csa.h).
+constexpr uint32_t CSA_DEV_OK = 0;
+constexpr uint32_t CSA_DEV_TIMEOUT = 4;
+constexpr uint32_t CSA_DEV_BOUNDS = 6;
+
+// A bounded wait gives up after this many SM clock cycles (about half a second at the
+// B200's clocks), records CSA_DEV_TIMEOUT and lets the kernel unwind.
+constexpr long long kWaitCycles = 1ll << 30;
+
+// The status word lives in the first 256 bytes of every workspace.
+constexpr size_t kStatusBytes = 256;
+
+// Debugging builds (-DCSA_TRACE) may place the workspace in host-mapped memory, where device
+// atomics are not available on every platform: they use plain stores instead.
+__device__ __forceinline__ void record_status(uint32_t* status, uint32_t code) {
+#ifdef CSA_TRACE
+  if (status != nullptr) *reinterpret_cast<volatile uint32_t*>(status) = code;
+#else
+  if (status != nullptr) atomicCAS(status, CSA_DEV_OK, code);
+#endif
+}
+
+// Where a bounded wait gave up (first one wins): status word 1.
+__device__ __forceinline__ void record_site(uint32_t* status, uint32_t site) {
+#ifdef CSA_TRACE
+  if (status != nullptr) *reinterpret_cast<volatile uint32_t*>(status + 1) = site;
+#else
+  if (status != nullptr) atomicCAS(status + 1, 0u, site);
+#endif
+}
+
+// Progress markers for debugging builds (-DCSA_TRACE): role `role` of the calling CTA stores `v`
+// into status word 64 + 4*cta + role. Compiled out otherwise.
+__device__ __forceinline__ void trace_mark(uint32_t* status, int role, uint32_t v) {
+#ifdef CSA_TRACE
+  if (status != nullptr) {
+    const uint32_t cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    volatile uint32_t* p = status + 64 + 4 * cta + role;
+    *p = v;
+  }
+#else
+  (void)status;
+  (void)role;
+  (void)v;
+#endif
+}
+
+// Timeline for debugging builds (-DCSA_TRACE): CTA (0,0) stores the low word of %globaltimer (ns)
+// into status word 1024 + idx. Compiled out otherwise.
+__device__ __forceinline__ void trace_time(uint32_t* status, int idx) {
+#ifdef CSA_TRACE
+  if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
+    uint32_t t;
+    asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
+    *reinterpret_cast<volatile uint32_t*>(status + 1024 + idx) = t;
+  }
+#else
+  (void)status;
+  (void)idx;
+#endif
+}
+
+}  // namespace csa

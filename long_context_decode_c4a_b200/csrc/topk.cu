@@ -1,0 +1,254 @@
+// topk.cu -- top-k selection of the lightning indexer's scores (K3).
+//
+// "DeepSeek-V4-Pro 架构：一个 token 的旅程", section "少读 KV 之前，Indexer 仍要给历史打分": top-k fixes
+// the main attention reads; "图解DeepSeek V4：详细计算流程解析" §2.2: the index module outputs the
+// indices of <= topK compressed entries. Ties go to the lower index; the output lists the chosen
+// indices in ascending order, padded with -1.
+//
+// Method: block-level radix select on order-preserving 32-bit keys (8 bits per pass, MSB first)
+// finds the k-th largest key T and how many keys equal to T to keep; a compaction pass in index
+// order then keeps every key > T and the first `need` keys == T. Inputs of up to kSmemKeys
+// entries are staged once in shared memory; longer score rows are cut into chunks whose local
+// top-k lists (in index order) are merged by a second launch with the same routine. The global
+// order (score desc, index asc) restricted to a chunk is the chunk's own order, so the global
+// top-k is contained in the union of the chunks' top-k lists.
+
+#include "kernels.cuh"
+
+namespace csa {
+
+namespace {
+
+// Order-preserving key: larger score -> larger key; -0 == +0; NaN below every number.
+__device__ __forceinline__ uint32_t score_key(float f) {
+  if (f != f) return 0u;
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+struct TopkShared {
+  uint32_t hist[256];
+  uint32_t warp_tot[32][2];
+  uint32_t digit, above, total;
+};
+
+// Exclusive prefix of two per-thread counts across the block (thread order), and the totals.
+__device__ __forceinline__ void block_scan2(uint32_t a, uint32_t b, TopkShared& sh, uint32_t& pre_a, uint32_t& pre_b,
+                                            uint32_t& tot_a, uint32_t& tot_b) {
+  const uint32_t lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  uint32_t ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t ya = __shfl_up_sync(0xffffffffu, ia, o);
+    const uint32_t yb = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= (uint32_t)o) {
+      ia += ya;
+      ib += yb;
+    }
+  }
+  __syncthreads();
+  if (lane == 31) {
+    sh.warp_tot[w][0] = ia;
+    sh.warp_tot[w][1] = ib;
+  }
+  __syncthreads();
+  uint32_t oa = 0, ob = 0, ta = 0, tb = 0;
+  for (uint32_t i = 0; i < nw; ++i) {
+    const uint32_t xa = sh.warp_tot[i][0], xb = sh.warp_tot[i][1];
+    if (i < w) {
+      oa += xa;
+      ob += xb;
+    }
+    ta += xa;
+    tb += xb;
+  }
+  pre_a = oa + ia - a;
+  pre_b = ob + ib - b;
+  tot_a = ta;
+  tot_b = tb;
+}
+
+// Select the top k of n keys (key(i), valid(i)) with ties to the lower position, and call
+// emit(pos, i) for the chosen positions in increasing i (pos = 0, 1, ...). Returns the count.
+// Each thread owns the contiguous positions [tid*per, tid*per + per).
+template <class KeyFn, class EmitFn>
+__device__ uint32_t block_topk(int n, int k, KeyFn key_of, EmitFn emit, TopkShared& sh) {
+  const int tid = threadIdx.x;
+  const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  // Count valid entries.
+  uint32_t cnt = 0;
+  for (int i = lo; i < hi; ++i) {
+    bool v;
+    (void)key_of(i, v);
+    cnt += v ? 1u : 0u;
+  }
+  {
+    uint32_t pa, pb, ta, tb;
+    block_scan2(cnt, 0u, sh, pa, pb, ta, tb);
+    cnt = ta;
+  }
+  const bool take_all = (int)cnt <= k;
+  uint32_t prefix = 0, mask = 0;
+  int krem = k;
+  if (!take_all) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += blockDim.x) sh.hist[i] = 0;
+      __syncthreads();
+      // Warp-aggregated histogram: lanes holding the same digit add once.
+      for (int r = 0; r < per; ++r) {
+        const int i = lo + r;
+        bool v = false;
+        uint32_t key = 0;
+        if (i < hi) key = key_of(i, v);
+        const bool live = v && (key & mask) == prefix;
+        const uint32_t dig = live ? ((key >> shift) & 255u) : 256u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+        if (live && (__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+      }
+      __syncthreads();
+      if (tid < 32) {
+        // lane L owns bins 255-8L .. 248-8L (descending); find the bin where the count of keys
+        // with a larger digit first reaches krem.
+        uint32_t loc[8];
+        uint32_t s = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          loc[j] = sh.hist[255 - 8 * tid - j];
+          s += loc[j];
+        }
+        uint32_t incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += y;
+        }
+        const uint32_t excl = incl - s;
+        if (excl < (uint32_t)krem && incl >= (uint32_t)krem) {
+          uint32_t run = excl;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (run + loc[j] >= (uint32_t)krem) {
+              sh.digit = 255 - 8 * tid - j;
+              sh.above = run;
+              break;
+            }
+            run += loc[j];
+          }
+        }
+      }
+      __syncthreads();
+      krem -= (int)sh.above;
+      prefix |= sh.digit << shift;
+      mask |= 0xFFu << shift;
+    }
+  }
+  // Compaction in index order: keep every key > T and the first `need` keys == T.
+  const uint32_t T = prefix;
+  const uint32_t need = take_all ? 0u : (uint32_t)krem;
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int i = lo; i < hi; ++i) {
+    bool v;
+    const uint32_t key = key_of(i, v);
+    if (!v) continue;
+    if (take_all || key > T) ++n_gt;
+    else if (key == T) ++n_eq;
+  }
+  uint32_t pre_gt, pre_eq, tot_gt, tot_eq;
+  block_scan2(n_gt, n_eq, sh, pre_gt, pre_eq, tot_gt, tot_eq);
+  uint32_t eq_seen = pre_eq;                            // keys == T before this thread's range
+  uint32_t pos = pre_gt + min(pre_eq, need);            // output slot of the next selected key
+  for (int i = lo; i < hi; ++i) {
+    bool v;
+    const uint32_t key = key_of(i, v);
+    if (!v) continue;
+    if (take_all || key > T) {
+      emit(pos++, i);
+    } else if (key == T) {
+      if (eq_seen < need) emit(pos++, i);
+      ++eq_seen;
+    }
+  }
+  return tot_gt + min(tot_eq, need);
+}
+
+}  // namespace
+
+// One CTA per (query, chunk). Chunk c of query q covers entries [c*chunk, min(E, (c+1)*chunk)).
+// Single-chunk queries write the final list; otherwise the chunk's top-k (key, index) pairs go to
+// the candidate buffers for topk_merge_kernel.
+__global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  __shared__ TopkShared sh;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);
+  const int q = blockIdx.y;
+  const int c = blockIdx.x;
+  const int t = P.q_pos[q];
+  int E = (t + 1) / P.ratio;
+  if (E > P.max_entries) {
+    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    E = P.max_entries;
+  }
+  if (E < 0) E = 0;
+  const int nchunks = (E + P.chunk - 1) / P.chunk;
+  const int lo = c * P.chunk;
+  const int n = max(0, min(E - lo, P.chunk));
+  int32_t* out = P.out + (long long)q * P.topk;
+  if (nchunks <= 1) {
+    if (c != 0) return;
+  } else if (c >= nchunks) {
+    // No entries here: mark the slot empty for the merge.
+    if (threadIdx.x == 0) P.cand_cnt[(long long)q * P.max_chunks + c] = 0;
+    return;
+  }
+  const float* row = P.scores + (long long)q * P.scores_stride + lo;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = score_key(row[i]);
+  __syncthreads();
+  auto key_of = [&](int i, bool& v) -> uint32_t {
+    v = true;
+    return keys[i];
+  };
+  if (nchunks <= 1) {
+    const uint32_t cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = lo + i; }, sh);
+    for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
+  } else {
+    const long long cb = ((long long)q * P.max_chunks + c) * P.topk;
+    uint32_t* ck = P.cand_key + cb;
+    int32_t* ci = P.cand_idx + cb;
+    const uint32_t cnt =
+        block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { ck[pos] = keys[i]; ci[pos] = lo + i; }, sh);
+    if (threadIdx.x == 0) P.cand_cnt[(long long)q * P.max_chunks + c] = (int)cnt;
+  }
+}
+
+// One CTA per query with more than one chunk: top-k over the union of the chunks' lists. The
+// lists are in ascending index order and chunk order is index order, so position order in the
+// concatenation is index order (unused slots are marked invalid).
+__global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) {
+  __shared__ TopkShared sh;
+  __shared__ int cnts[kTopkMaxChunks];
+  const int q = blockIdx.x;
+  const int t = P.q_pos[q];
+  int E = (t + 1) / P.ratio;
+  if (E > P.max_entries) E = P.max_entries;
+  if (E < 0) E = 0;
+  const int nchunks = (E + P.chunk - 1) / P.chunk;
+  if (nchunks <= 1) return;
+  for (int c = threadIdx.x; c < nchunks; c += blockDim.x) cnts[c] = P.cand_cnt[(long long)q * P.max_chunks + c];
+  __syncthreads();
+  const long long cb = (long long)q * P.max_chunks * P.topk;
+  const uint32_t* ck = P.cand_key + cb;
+  const int32_t* ci = P.cand_idx + cb;
+  const int n = nchunks * P.topk;
+  const int K = P.topk;
+  auto key_of = [&](int i, bool& v) -> uint32_t {
+    v = (i % K) < cnts[i / K];
+    return v ? ck[i] : 0u;
+  };
+  int32_t* out = P.out + (long long)q * P.topk;
+  const uint32_t cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = ci[i]; }, sh);
+  for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
+}
+
+}  // namespace csa

@@ -1,0 +1,128 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol include/csa.h declares,
+matches the header's struct layouts, and rejects bad arguments on the host before any launch."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from long_context_decode_c4a_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^CSA_API\s+[\w\s\*]+?\b((?:csa|hca)_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_symbols()
+    for want in ("csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode_fused",
+                 "hca_decode_fused", "csa_workspace_size", "csa_get_device_status", "csa_state_reset"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\sT\s(\w+)$", out, flags=re.M))
+    for name in declared_symbols():
+        assert name in exported, name
+        assert hasattr(lib, name)
+    assert set(_lib.PROTOTYPES) == set(declared_symbols())
+
+
+def _c_offsets(struct, fields):
+    prog = "#include <stdio.h>\n#include <stddef.h>\n#include \"csa.h\"\nint main(void){\n"
+    prog += f'printf("%zu\\n", sizeof({struct}));\n'
+    for f in fields:
+        prog += f'printf("%zu\\n", offsetof({struct}, {f}));\n'
+    prog += "return 0;}\n"
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(prog)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()]
+    return vals[0], vals[1:]
+
+
+@pytest.mark.parametrize("cls,cname", [(_lib.DecodeArgs, "csa_decode_args"), (_lib.HcaDecodeArgs, "hca_decode_args"),
+                                       (_lib.CompressorCfg, "csa_compressor_cfg")])
+def test_struct_layout_matches_header(cls, cname):
+    fields = [f for f, _ in cls._fields_]
+    size, offs = _c_offsets(cname, fields)
+    assert ctypes.sizeof(cls) == size
+    for (f, _), o in zip(cls._fields_, offs):
+        assert getattr(cls, f).offset == o, f
+
+
+def test_status_strings_and_version(lib):
+    assert lib.csa_version() == 1
+    for code in range(7):
+        assert lib.csa_status_string(code)
+    assert lib.csa_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    n = ctypes.c_size_t()
+    assert lib.csa_workspace_size(_lib.CSA_WS_DECODE_FUSED, 64, 1, 8192, 1024, ctypes.byref(n)) == 0
+    assert n.value >= 256 + 64 * 8192 * 4 and n.value % 256 == 0
+    assert lib.csa_workspace_size(_lib.CSA_WS_INDEXER_TOPK, 8, 1, 262144, 1024, ctypes.byref(n)) == 0
+    # long rows need the chunked top-k lists: 16 chunks x 1024 (key, index) pairs per query
+    assert n.value >= 256 + 8 * 262144 * 4 + 2 * 8 * 16 * 1024 * 4
+    assert lib.csa_workspace_size(_lib.CSA_WS_HCA_ATTN, 64, 1, 256, 0, ctypes.byref(n)) == 0
+    assert n.value == 256
+    assert lib.csa_workspace_size(99, 1, 1, 1, 1, ctypes.byref(n)) == _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_workspace_size(_lib.CSA_WS_DECODE_FUSED, 0, 1, 1, 1, ctypes.byref(n)) == _lib.CSA_ERR_INVALID_ARG
+
+
+def test_host_side_argument_checks_launch_nothing(lib):
+    """Every bad argument is rejected before any CUDA call (this host has no GPU)."""
+    cfg = _lib.CompressorCfg(4, 1, 512, 64, 10000.0, 1e-6)
+    null = None
+    # null pointers
+    rc = lib.csa_compress(ctypes.byref(cfg), 1, 4, null, null, null, null, null, null, null, 4096, 8, null, null)
+    assert rc == _lib.CSA_ERR_INVALID_ARG
+    # unsupported compressor configuration
+    bad = _lib.CompressorCfg(8, 1, 512, 64, 10000.0, 1e-6)
+    assert lib.csa_compress(ctypes.byref(bad), 1, 4, 16, 16, 16, 16, 16, 16, 16, 4096, 8, null, null) == \
+        _lib.CSA_ERR_UNSUPPORTED
+    # misaligned pointer (8-byte aligned, not 16)
+    assert lib.csa_compress(ctypes.byref(cfg), 1, 4, 16, 24, 16, 16, 16, 16, 16, 4096, 8, null, null) == \
+        _lib.CSA_ERR_INVALID_ARG
+    # indexer: d_I must be 128, H_I a power of two
+    assert lib.csa_indexer_topk(1, 1, 64, 64, 4, 8, 16, 16, 16, 16, 64 * 8, 8, 16, null, 256, 4096, null) == \
+        _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_indexer_topk(1, 1, 48, 128, 4, 8, 16, 16, 16, 16, 128 * 8, 8, 16, null, 256, 4096, null) == \
+        _lib.CSA_ERR_UNSUPPORTED
+    # indexer: topk over the supported maximum
+    assert lib.csa_indexer_topk(1, 1, 64, 128, 4, 4096, 16, 16, 16, 16, 128 * 8, 8, 16, null, 256, 4096, null) == \
+        _lib.CSA_ERR_UNSUPPORTED
+    # attention: d must be 512, window <= ring_cap, workspace present
+    assert lib.csa_sparse_attn(1, 1, 128, 256, 64, 1e4, 0.05, 16, 16, 16, 256 * 128, 128, 128, 16, 256 * 8, 8, 16,
+                               8, 16, 16, 0, 256, 256, null) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_sparse_attn(1, 1, 128, 512, 64, 1e4, 0.05, 16, 16, 16, 512 * 64, 64, 128, 16, 512 * 8, 8, 16,
+                               8, 16, 16, 0, 256, 256, null) == _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_sparse_attn(1, 1, 128, 512, 64, 1e4, 0.05, 16, 16, 16, 512 * 128, 128, 128, 16, 512 * 8, 8, 16,
+                               8, 16, 16, 0, null, 0, null) == _lib.CSA_ERR_WORKSPACE
+    # attention: ring stride not a multiple of d
+    assert lib.hca_attn(1, 1, 128, 512, 64, 1e4, 0.05, 128, 16, 16, 16, 512 * 128 + 8, 128, 128, 16, 512 * 8, 8, 16,
+                        16, 0, 256, 256, null) == _lib.CSA_ERR_INVALID_ARG
+    # fused decode: null args
+    assert lib.csa_decode_fused(None, null) == _lib.CSA_ERR_INVALID_ARG
+    a = _lib.DecodeArgs()
+    a.B, a.ratio = 1, 4
+    assert lib.csa_decode_fused(ctypes.byref(a), null) in (_lib.CSA_ERR_INVALID_ARG, _lib.CSA_ERR_UNSUPPORTED)
+    st = ctypes.c_int()
+    assert lib.csa_get_device_status(None, null, ctypes.byref(st)) == _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_last_error()

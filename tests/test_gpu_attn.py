@@ -1,0 +1,152 @@
+"""GPU parity of sparse MQA with sink + inverse RoPE (csa_sparse_attn) and HCA attention (hca_attn)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import csa_oracle as O
+from tests.parity import assert_attn_close, np64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ops():
+    from long_context_decode_c4a_b200 import ops
+    return ops
+
+
+def _q(B, S, H, d, g):
+    x = torch.randn(B, S, H, d, generator=g)
+    return (x * torch.rsqrt(x.square().mean(-1, keepdim=True) + 1e-6)).to(torch.bfloat16)
+
+
+def _random_topk(B, S, pos, k, ratio, g):
+    out = torch.full((B, S, k), -1, dtype=torch.int32)
+    for b in range(B):
+        for i in range(S):
+            E = (int(pos[b, i]) + 1) // ratio
+            n = min(k, E)
+            if n:
+                sel = torch.randperm(E, generator=g)[:n].sort().values
+                out[b, i, :n] = sel.to(torch.int32)
+    return out
+
+
+@pytest.mark.parametrize("case", ["decode", "early_positions", "tiny_heads", "bf16_out"])
+def test_sparse_attn(ops, case):
+    g = torch.Generator().manual_seed(hash(case) % 997)
+    d = 512
+    if case == "decode":
+        B, S, H, W, k, E_cap = 3, 1, 128, 128, 1024, 8192
+        pos = torch.tensor([[32767], [20001], [4200]], dtype=torch.int32)
+        ring_cap = W
+    elif case == "early_positions":   # t < window and t < 3: partial window, no or few entries
+        B, S, H, W, k, E_cap = 1, 6, 128, 128, 64, 64
+        pos = torch.tensor([[0, 1, 3, 5, 100, 255]], dtype=torch.int32)
+        ring_cap = 256
+    elif case == "tiny_heads":
+        B, S, H, W, k, E_cap = 1, 4, 8, 16, 8, 32
+        pos = torch.tensor([[17, 64, 100, 127]], dtype=torch.int32)
+        ring_cap = 128
+    else:
+        B, S, H, W, k, E_cap = 2, 1, 128, 128, 200, 1000
+        pos = torch.tensor([[3999], [777]], dtype=torch.int32)
+        ring_cap = W
+    q = _q(B, S, H, d, g)
+    ring = torch.randn(B, ring_cap, d, generator=g).to(torch.bfloat16)
+    cache = torch.randn(B, E_cap, d, generator=g).to(torch.bfloat16)
+    sink = torch.randn(H, generator=g)
+    topk = _random_topk(B, S, pos, k, 4, g)
+    out_dtype = torch.bfloat16 if case == "bf16_out" else torch.float32
+    out = torch.empty(B, S, H, d, dtype=out_dtype, device="cuda")
+    ops.sparse_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), topk.cuda(), sink.cuda(), W, out=out)
+    torch.cuda.synchronize()
+    for b in range(B):
+        for i in range(S):
+            t = int(pos[b, i])
+            ref = O.attend_query(np64(q[b, i]), t, W, np64(ring[b]), ring_cap, np64(cache[b]),
+                                 np64(topk[b, i]).tolist(), np64(sink), 1 / math.sqrt(d), 64, 10000.0)
+            assert_attn_close(out[b, i], ref, f"{case} b={b} i={i} t={t}", bf16_out=out_dtype == torch.bfloat16)
+
+
+def test_sink_minus_infinity_is_plain_softmax(ops):
+    """T6 on the GPU: a sink of -inf removes the sink term."""
+    g = torch.Generator().manual_seed(3)
+    B, S, H, d, W = 1, 1, 128, 512, 128
+    pos = torch.tensor([[999]], dtype=torch.int32)
+    q = _q(B, S, H, d, g)
+    ring = torch.randn(B, W, d, generator=g).to(torch.bfloat16)
+    cache = torch.randn(B, 250, d, generator=g).to(torch.bfloat16)
+    topk = _random_topk(B, S, pos, 100, 4, g)
+    sink = torch.full((H,), float("-inf"))
+    out = torch.empty(B, S, H, d, dtype=torch.float32, device="cuda")
+    ops.sparse_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), topk.cuda(), sink.cuda(), W, out=out)
+    torch.cuda.synchronize()
+    ref = O.attend_query(np64(q[0, 0]), 999, W, np64(ring[0]), W, np64(cache[0]), np64(topk[0, 0]).tolist(),
+                         np64(sink), 1 / math.sqrt(d), 64, 10000.0)
+    assert np.all(np.isfinite(ref))
+    assert_attn_close(out[0, 0], ref, "sink -inf")
+
+
+def test_large_logits_rescale(ops):
+    """Candidates whose logits jump far above the running max force the O rescale path."""
+    g = torch.Generator().manual_seed(4)
+    B, S, H, d, W = 1, 1, 128, 512, 128
+    pos = torch.tensor([[4095]], dtype=torch.int32)
+    q = _q(B, S, H, d, g)
+    ring = torch.randn(B, W, d, generator=g).to(torch.bfloat16)
+    cache = torch.randn(B, 1024, d, generator=g).to(torch.bfloat16)
+    # late entries aligned with q (per head 0 direction) produce logits ~ +20 in later tiles
+    cache[0, 900:] = (q[0, 0, 0].float() * 6).to(torch.bfloat16)
+    topk = torch.arange(1024, dtype=torch.int32).reshape(1, 1, 1024)
+    sink = torch.zeros(H)
+    out = torch.empty(B, S, H, d, dtype=torch.float32, device="cuda")
+    ops.sparse_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), topk.cuda(), sink.cuda(), W, out=out)
+    torch.cuda.synchronize()
+    ref = O.attend_query(np64(q[0, 0]), 4095, W, np64(ring[0]), W, np64(cache[0]), list(range(1024)), np64(sink),
+                         1 / math.sqrt(d), 64, 10000.0)
+    assert_attn_close(out[0, 0], ref, "rescale")
+
+
+@pytest.mark.parametrize("ratio,E_cap,pos_list", [(128, 256, [32767, 20000, 127, 5000]), (4, 600, [2399, 130])])
+def test_hca_attn(ops, ratio, E_cap, pos_list):
+    g = torch.Generator().manual_seed(ratio)
+    B, S, H, d, W = len(pos_list), 1, 128, 512, 128
+    pos = torch.tensor(pos_list, dtype=torch.int32)[:, None]
+    q = _q(B, S, H, d, g)
+    ring = torch.randn(B, W, d, generator=g).to(torch.bfloat16)
+    cache = torch.randn(B, E_cap, d, generator=g).to(torch.bfloat16)
+    sink = torch.randn(H, generator=g)
+    out = torch.empty(B, S, H, d, dtype=torch.float32, device="cuda")
+    ops.hca_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), sink.cuda(), W, ratio=ratio, out=out)
+    torch.cuda.synchronize()
+    for b in range(B):
+        t = pos_list[b]
+        vis = min((t + 1) // ratio, E_cap)
+        ref = O.attend_query(np64(q[b, 0]), t, W, np64(ring[b]), W, np64(cache[b]), list(range(vis)), np64(sink),
+                             1 / math.sqrt(d), 64, 10000.0)
+        assert_attn_close(out[b, 0], ref, f"hca b={b} t={t}")
+
+
+def test_csa_with_all_entries_equals_hca(ops):
+    """T5 on the GPU: top-k covering every visible entry gives the HCA (dense) result."""
+    g = torch.Generator().manual_seed(9)
+    B, S, H, d, W = 2, 1, 128, 512, 128
+    pos = torch.tensor([[1023], [555]], dtype=torch.int32)
+    q = _q(B, S, H, d, g)
+    ring = torch.randn(B, W, d, generator=g).to(torch.bfloat16)
+    cache = torch.randn(B, 256, d, generator=g).to(torch.bfloat16)
+    sink = torch.randn(H, generator=g)
+    topk = torch.full((B, S, 300), -1, dtype=torch.int32)
+    for b in range(B):
+        E = (int(pos[b, 0]) + 1) // 4
+        topk[b, 0, :E] = torch.arange(E, dtype=torch.int32)
+    o1 = torch.empty(B, S, H, d, dtype=torch.float32, device="cuda")
+    o2 = torch.empty_like(o1)
+    ops.sparse_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), topk.cuda(), sink.cuda(), W, out=o1)
+    ops.hca_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), sink.cuda(), W, ratio=4, out=o2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
