@@ -114,7 +114,6 @@ int device_info(DeviceInfo** out) {
     CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
     CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
     CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
-    CSA_CUDA(cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTopkChunk * 4));
     d.attrs_set = true;
   }
   *out = &d;
@@ -278,8 +277,9 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
   while (stages > 2 && indexer_smem_bytes(stages, P.N) > (size_t)dev->max_smem) --stages;
   CSA_CHECK_SUP(indexer_smem_bytes(stages, P.N) <= (size_t)dev->max_smem, "shared memory too small for the indexer");
   P.stages = stages;
+  P.n_acc = (4 * P.N <= 512) ? 4 : 2;
   int cols = 32;
-  while (cols < 2 * P.N) cols <<= 1;
+  while (cols < P.n_acc * P.N) cols <<= 1;
   P.tmem_cols = cols;
   P.q_pos = a.q_pos;
   P.w = a.w;
@@ -318,8 +318,7 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
   T.cand_cnt = reinterpret_cast<int*>(ws + L.cand_cnt_off);
   T.status = status;
   const int nchunks = std::max(1, L.max_chunks);
-  const size_t tsmem = (size_t)std::min(a.max_entries, kTopkChunk) * 4;
-  topk_chunk_kernel<<<dim3((unsigned)nchunks, (unsigned)queries), kTopkThreads, tsmem, st>>>(T);
+  topk_chunk_kernel<<<dim3((unsigned)nchunks, (unsigned)queries), kTopkThreads, 0, st>>>(T);
   CSA_CUDA(cudaGetLastError());
   if (L.max_chunks > 1) {
     CSA_CHECK_SUP(L.max_chunks <= kTopkMaxChunks, "max_entries too large for the top-k merge");

@@ -163,6 +163,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaun
   const int tid = threadIdx.x;
   const bool active = tid < d / 8;
   const int c0 = tid * 8;
+  if (tid == 0) trace_time(P.status, 512);
 
   // Window-ring write of the fused decode step (main stream only).
   if (P.win_src != nullptr && blockIdx.x == 0) {
@@ -173,6 +174,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaun
       *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<const uint4*>(src + c);
   }
 
+  if (tid == 0) trace_time(P.status, 513);
   if (g <= g_last) {
     if (g >= P.max_entries) {
       if (tid == 0) record_status(P.status, CSA_DEV_BOUNDS);
@@ -235,6 +237,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaun
           }
         }
       }
+      if (tid == 0) trace_time(P.status, 514);
       float x[8];
       float ss = 0.f;
 #pragma unroll
@@ -243,6 +246,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaun
         ss += x[i] * x[i];
       }
       const float tot = block_sum(ss, red);
+      if (tid == 0) trace_time(P.status, 515);
       const float r = rsqrtf(tot / (float)d + P.eps);
       // RoPE table for position g*ratio: the angle is formed in double precision.
       const int npairs = P.rope_dim / 2;
@@ -254,6 +258,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaun
         rope_cs[2 * tid + 1] = sn;
       }
       __syncthreads();
+      if (tid == 0) trace_time(P.status, 516);
       if (active) {
         const Vec8 gm = load8(P.gamma + c0);
         float y[8];
@@ -286,10 +291,12 @@ __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaun
     }
   }
 
+  if (tid == 0) trace_time(P.status, 517);
   if (P.fuse_state && blockIdx.x == 0) {
     __syncthreads();
     update_state(P, b, start, end);
   }
+  if (tid == 0) trace_time(P.status, 518);
 }
 
 // Final state of a multi-token segment: one CTA per request, reads before writes.

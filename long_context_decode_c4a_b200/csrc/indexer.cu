@@ -76,17 +76,17 @@ struct ItemIter {
 struct IdxSmem {
   uint64_t k_full[kIdxMaxStages], k_empty[kIdxMaxStages];
   uint64_t q_full[2], q_empty[2];
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t acc_full[4], acc_empty[4];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float w[256];
-  int vis[256];
+  float w[2][256];   // per epilogue group: w of the group's current queries
+  int vis[2][256];   // per epilogue group: visible entries of those queries
 };
 
 template <int HI>
-__device__ __forceinline__ void epilogue_tile(const IndexerParams& P, const IdxSmem& sm, uint32_t tmem_acc, int b,
-                                              int qg, int et, int row) {
+__device__ __forceinline__ void epilogue_tile(const IndexerParams& P, const float* w_s, const int* vis_s,
+                                              uint32_t tmem_acc, int b, int qg, int et, int row) {
   constexpr int kQPerChunk = HI >= 32 ? 1 : 32 / HI;
   constexpr int kChunksPerQ = HI >= 32 ? HI / 32 : 1;
   constexpr int kColsPerQ = HI >= 32 ? 32 : HI;
@@ -94,9 +94,12 @@ __device__ __forceinline__ void epilogue_tile(const IndexerParams& P, const IdxS
   const int s = et * 128 + row;
   const int ncols = nq * HI;
   for (int col0 = 0; col0 < ncols; col0 += 32 * kChunksPerQ) {
-    float sigma[kQPerChunk];
+    // Four independent partial sums per query keep the FMA chains short.
+    float part[kQPerChunk][4];
 #pragma unroll
-    for (int j = 0; j < kQPerChunk; ++j) sigma[j] = 0.f;
+    for (int j = 0; j < kQPerChunk; ++j)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) part[j][u] = 0.f;
 #pragma unroll
     for (int c = 0; c < kChunksPerQ; ++c) {
       uint32_t v[32];
@@ -105,15 +108,16 @@ __device__ __forceinline__ void epilogue_tile(const IndexerParams& P, const IdxS
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float x = __uint_as_float(v[j]);
-        sigma[j / kColsPerQ] = fmaf(sm.w[col0 + 32 * c + j], fmaxf(x, 0.f), sigma[j / kColsPerQ]);
+        float& acc = part[j / kColsPerQ][j & 3];
+        acc = fmaf(w_s[col0 + 32 * c + j], fmaxf(x, 0.f), acc);
       }
     }
 #pragma unroll
     for (int j = 0; j < kQPerChunk; ++j) {
       const int qi = col0 / HI + j;
-      if (qi < nq && s < sm.vis[qi]) {
+      if (qi < nq && s < vis_s[qi]) {
         const long long qrow = (long long)b * P.S + (long long)qg * P.QG + qi;
-        P.scores[qrow * P.scores_stride + s] = sigma[j];
+        P.scores[qrow * P.scores_stride + s] = (part[j][0] + part[j][1]) + (part[j][2] + part[j][3]);
       }
     }
   }
@@ -144,6 +148,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
+    }
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&sm.acc_full[i], 1);
       mbar_init(&sm.acc_empty[i], 128);
     }
@@ -155,7 +161,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     tma_prefetch_desc(&map_k);
     tma_prefetch_desc(&map_q);
   }
-  const uint32_t acc_cols = (uint32_t)P.tmem_cols;  // power of two >= 2N
+  const uint32_t acc_cols = (uint32_t)P.tmem_cols;  // power of two >= n_acc * N
+  const int n_acc = P.n_acc;                         // 2 or 4 accumulators (even: one parity per group)
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, acc_cols);
     tmem_relinquish();
@@ -218,8 +225,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         const int st = (int)(n % NS);
         if (!mbar_wait(&sm.k_full[st], (uint32_t)((n / NS) & 1), abort_flag, status, 212)) break;
-        const int a = (int)(n & 1);
-        if (!mbar_wait(&sm.acc_empty[a], (uint32_t)(((n >> 1) & 1) ^ 1), abort_flag, status, 213)) break;
+        const int a = (int)(n % n_acc);
+        if (!mbar_wait(&sm.acc_empty[a], (uint32_t)(((n / n_acc) & 1) ^ 1), abort_flag, status, 213)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(a * N);
         const uint32_t ka = smem_u32(k_tiles + (size_t)st * 32768);
@@ -242,31 +249,40 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       trace_mark(status, 1, 9);
     }
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 2..5)
-    const int et_tid = threadIdx.x - 64;              // 0..127
+    // ---------------------------------------------------------------- epilogue (warps 2..9)
+    // Two groups of four warps take alternate work items (group g: items n with n % 2 == g), each
+    // group covering the four TMEM lane quadrants.
+    const int grp = (warp - 2) >> 2;
+    const int gt = threadIdx.x - 64 - 128 * grp;      // 0..127 within the group
     const int quad = warp & 3;                        // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
+    float* w_s = sm.w[grp];
+    int* vis_s = sm.vis[grp];
     ItemIter iter(it0, it1);
     ItemCoord c;
     bool ng;
     long long n = 0;
+    int cur_b = -1, cur_qg = -1;
     while (iter.next(P, c, ng)) {
-      if (ng) {
-        named_bar_sync(1, 128);
+      const long long my = n++;
+      if ((my & 1) != grp) continue;
+      if (c.b != cur_b || c.qg != cur_qg) {
+        named_bar_sync(1 + 2 * grp, 128);
         const int nq = min(P.QG, P.S - c.qg * P.QG);
         const long long q0 = (long long)c.b * P.S + (long long)c.qg * P.QG;
-        for (int j = et_tid; j < nq * HI; j += 128) sm.w[j] = P.w[q0 * HI + j];
-        for (int j = et_tid; j < nq; j += 128) sm.vis[j] = visible_of(P, c.b, c.qg * P.QG + j);
-        named_bar_sync(1, 128);
+        for (int j = gt; j < nq * HI; j += 128) w_s[j] = P.w[q0 * HI + j];
+        for (int j = gt; j < nq; j += 128) vis_s[j] = visible_of(P, c.b, c.qg * P.QG + j);
+        named_bar_sync(1 + 2 * grp, 128);
+        cur_b = c.b;
+        cur_qg = c.qg;
       }
-      const int a = (int)(n & 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full[a], (uint32_t)((n >> 1) & 1), abort_flag, status, 221))) break;
-      if (et_tid == 0) trace_mark(status, 2, (uint32_t)(100 + n));
+      const int a = (int)(my % n_acc);
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full[a], (uint32_t)((my / n_acc) & 1), abort_flag, status, 221))) break;
+      if (gt == 0) trace_mark(status, 2, (uint32_t)(100 + my));
       tc_fence_after();
-      epilogue_tile<HI>(P, sm, tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * N), c.b, c.qg, c.et, row);
+      epilogue_tile<HI>(P, w_s, vis_s, tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * N), c.b, c.qg, c.et, row);
       tc_fence_before();
       mbar_arrive(&sm.acc_empty[a]);
-      ++n;
     }
   }
   __syncwarp();

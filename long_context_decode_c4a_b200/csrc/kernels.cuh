@@ -51,7 +51,7 @@ __global__ void state_reset_kernel(uint16_t* kv, uint16_t* score, long long n);
 
 // ------------------------------------------------------------------------------ indexer (K2)
 
-constexpr int kIdxThreads = 192;          // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr int kIdxThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue (2 groups)
 constexpr int kIdxMaxStages = 8;
 
 struct IndexerParams {
@@ -62,7 +62,7 @@ struct IndexerParams {
   int groups_per_req, tiles_per_group;
   long long total_items;                  // B * groups_per_req * tiles_per_group
   long long rows_per_req;                 // index-cache rows per request (idx_bstride / d_I)
-  int stages, tmem_cols;
+  int stages, tmem_cols, n_acc;
   const int32_t* q_pos;                   // [B*S]
   const float* w;                         // [B*S, H_I]
   float* scores;                          // [B*S, scores_stride]

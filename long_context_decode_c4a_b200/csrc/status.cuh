@@ -53,13 +53,15 @@ __device__ __forceinline__ void trace_mark(uint32_t* status, int role, uint32_t 
 }
 
 // Timeline for debugging builds (-DCSA_TRACE): CTA (0,0) stores the low word of %globaltimer (ns)
-// into status word 1024 + idx. Compiled out otherwise.
+// into word kTraceWord + idx of the workspace (a debugging workspace of >= 8 MB). Compiled out
+// otherwise.
+constexpr size_t kTraceWord = size_t(1) << 20;
 __device__ __forceinline__ void trace_time(uint32_t* status, int idx) {
 #ifdef CSA_TRACE
   if (status != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {
     uint32_t t;
     asm volatile("mov.u32 %0, %%globaltimer_lo;" : "=r"(t));
-    *reinterpret_cast<volatile uint32_t*>(status + 1024 + idx) = t;
+    *reinterpret_cast<volatile uint32_t*>(status + kTraceWord + idx) = t;
   }
 #else
   (void)status;

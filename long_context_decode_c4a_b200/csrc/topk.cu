@@ -173,21 +173,159 @@ __device__ uint32_t block_topk(int n, int k, KeyFn key_of, EmitFn emit, TopkShar
   return tot_gt + min(tot_eq, need);
 }
 
+constexpr int kRegKeys = kTopkChunk / kTopkThreads;   // keys per thread in the chunk kernel (16)
+
+struct TopkRegShared {
+  uint32_t hist[256];
+  uint32_t cnt[kRegKeys][32][2];   // per (key slot, warp): count of keys > T, == T
+  uint32_t off[kRegKeys][32][2];   // exclusive prefix over warps
+  uint32_t base[kRegKeys][2];      // keys > T / == T in all earlier key slots
+  uint32_t red[32];
+  uint32_t digit, above, total;
+};
+
+// Top-k of up to kRegKeys * blockDim keys held in registers. Thread t holds the keys of positions
+// i = r * blockDim + t (r = 0 .. kRegKeys-1). Chosen positions are passed to emit(pos, r) with
+// pos = 0, 1, ... in increasing i. Returns the count.
+template <class EmitFn>
+__device__ uint32_t block_topk_regs(const uint32_t (&key)[kRegKeys], int n, int k, EmitFn emit, TopkRegShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  auto valid = [&](int r) { return r * (int)blockDim.x + tid < n; };
+  uint32_t cnt = 0;
+#pragma unroll
+  for (int r = 0; r < kRegKeys; ++r) cnt += valid(r) ? 1u : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) sh.red[w] = cnt;
+  __syncthreads();
+  uint32_t total = 0;
+  for (int i = 0; i < nw; ++i) total += sh.red[i];
+  const bool take_all = (int)total <= k;
+  uint32_t prefix = 0, mask = 0;
+  int krem = k;
+  if (!take_all) {
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = tid; i < 256; i += blockDim.x) sh.hist[i] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < kRegKeys; ++r) {
+        const bool live = valid(r) && (key[r] & mask) == prefix;
+        const uint32_t dig = live ? ((key[r] >> shift) & 255u) : 256u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, dig);
+        if (live && (__ffs(peers) - 1) == lane) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
+      }
+      __syncthreads();
+      if (tid < 32) {
+        uint32_t loc[8];
+        uint32_t s = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          loc[j] = sh.hist[255 - 8 * tid - j];
+          s += loc[j];
+        }
+        uint32_t incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (tid >= o) incl += y;
+        }
+        const uint32_t excl = incl - s;
+        if (excl < (uint32_t)krem && incl >= (uint32_t)krem) {
+          uint32_t run = excl;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (run + loc[j] >= (uint32_t)krem) {
+              sh.digit = 255 - 8 * tid - j;
+              sh.above = run;
+              break;
+            }
+            run += loc[j];
+          }
+        }
+      }
+      __syncthreads();
+      krem -= (int)sh.above;
+      prefix |= sh.digit << shift;
+      mask |= 0xFFu << shift;
+    }
+  }
+  // Compaction in index order: keep every key > T and the first `need` keys == T.
+  const uint32_t T = prefix;
+  const uint32_t need = take_all ? 0u : (uint32_t)krem;
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int r = 0; r < kRegKeys; ++r) {
+    const bool gt = valid(r) && (take_all || key[r] > T);
+    const bool eq = valid(r) && !take_all && key[r] == T;
+    const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
+    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) {
+      sh.cnt[r][w][0] = __popc(bgt);
+      sh.cnt[r][w][1] = __popc(beq);
+    }
+  }
+  __syncthreads();
+  if (w == 0) {
+    uint32_t run0 = 0, run1 = 0;
+    for (int r = 0; r < kRegKeys; ++r) {
+      uint32_t v0 = lane < nw ? sh.cnt[r][lane][0] : 0u, v1 = lane < nw ? sh.cnt[r][lane][1] : 0u;
+      uint32_t i0 = v0, i1 = v1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y0 = __shfl_up_sync(0xffffffffu, i0, o), y1 = __shfl_up_sync(0xffffffffu, i1, o);
+        if (lane >= o) {
+          i0 += y0;
+          i1 += y1;
+        }
+      }
+      if (lane < nw) {
+        sh.off[r][lane][0] = i0 - v0;
+        sh.off[r][lane][1] = i1 - v1;
+      }
+      if (lane == 0) {
+        sh.base[r][0] = run0;
+        sh.base[r][1] = run1;
+      }
+      run0 += __shfl_sync(0xffffffffu, i0, 31);
+      run1 += __shfl_sync(0xffffffffu, i1, 31);
+    }
+    if (lane == 0) {
+      sh.above = run0;   // keys > T
+      sh.total = run1;   // keys == T
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kRegKeys; ++r) {
+    const bool gt = valid(r) && (take_all || key[r] > T);
+    const bool eq = valid(r) && !take_all && key[r] == T;
+    const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
+    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
+    if (!(gt || eq)) continue;
+    const uint32_t gt_before = sh.base[r][0] + sh.off[r][w][0] + __popc(bgt & lt);
+    const uint32_t eq_before = sh.base[r][1] + sh.off[r][w][1] + __popc(beq & lt);
+    if (gt) {
+      emit(gt_before + min(eq_before, need), r);
+    } else if (eq_before < need) {
+      emit(gt_before + eq_before, r);
+    }
+  }
+  return sh.above + min(sh.total, need);
+}
+
 }  // namespace
 
 // One CTA per (query, chunk). Chunk c of query q covers entries [c*chunk, min(E, (c+1)*chunk)).
 // Single-chunk queries write the final list; otherwise the chunk's top-k (key, index) pairs go to
 // the candidate buffers for topk_merge_kernel.
 __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ TopkShared sh;
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);
+  __shared__ TopkRegShared sh;
   const int q = blockIdx.y;
   const int c = blockIdx.x;
   const int t = P.q_pos[q];
   int E = (t + 1) / P.ratio;
   if (E > P.max_entries) {
-    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    if (threadIdx.x == 0 && c == 0) record_status(P.status, CSA_DEV_BOUNDS);
     E = P.max_entries;
   }
   if (E < 0) E = 0;
@@ -203,21 +341,25 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
     return;
   }
   const float* row = P.scores + (long long)q * P.scores_stride + lo;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) keys[i] = score_key(row[i]);
-  __syncthreads();
-  auto key_of = [&](int i, bool& v) -> uint32_t {
-    v = true;
-    return keys[i];
-  };
+  uint32_t key[kRegKeys];
+#pragma unroll
+  for (int r = 0; r < kRegKeys; ++r) {
+    const int i = r * (int)blockDim.x + (int)threadIdx.x;
+    key[r] = i < n ? score_key(row[i]) : 0u;
+  }
   if (nchunks <= 1) {
-    const uint32_t cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = lo + i; }, sh);
+    const uint32_t cnt = block_topk_regs(key, n, P.topk, [&](uint32_t pos, int r) {
+      out[pos] = lo + r * (int)blockDim.x + (int)threadIdx.x;
+    }, sh);
     for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
   } else {
     const long long cb = ((long long)q * P.max_chunks + c) * P.topk;
     uint32_t* ck = P.cand_key + cb;
     int32_t* ci = P.cand_idx + cb;
-    const uint32_t cnt =
-        block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { ck[pos] = keys[i]; ci[pos] = lo + i; }, sh);
+    const uint32_t cnt = block_topk_regs(key, n, P.topk, [&](uint32_t pos, int r) {
+      ck[pos] = key[r];
+      ci[pos] = lo + r * (int)blockDim.x + (int)threadIdx.x;
+    }, sh);
     if (threadIdx.x == 0) P.cand_cnt[(long long)q * P.max_chunks + c] = (int)cnt;
   }
 }

@@ -210,6 +210,9 @@ def _event_array(events, n: int):
         return None
     if len(events) != n:
         raise ValueError(f"stage_events needs {n} events")
+    for e in events:
+        if not e.cuda_event:      # torch creates the CUDA event on its first record
+            e.record()
     return (ctypes.c_void_p * n)(*[e.cuda_event for e in events])
 
 
