@@ -278,6 +278,25 @@ typedef struct {
 CSA_API int hca_decode_fused(const hca_decode_args* a, void* stream);
 
 /*
+ * csa_indexer_topk_noalloc -- csa_indexer_topk for callers that cannot allocate device memory (no
+ * counterpart in the pages; it is a deployment convenience). Such callers include code running
+ * inside another framework's memory pool without access to its allocator, plugins that are handed
+ * only the tensors they read and write, and paths that must never call cudaMalloc. Instead of a
+ * workspace it uses one fixed scratch array (4 MiB + 256 bytes) that the library defines in device
+ * memory; every GPU that loads the library holds it until the process exits. Arguments and
+ * results are those of csa_indexer_topk, without scores_opt and ws.
+ * Limits: max_entries <= 16384 and B*S*max_entries <= 1,048,576; larger calls return
+ * CSA_ERR_UNSUPPORTED without launching.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress), so
+ * make that first call before any stream capture on that device. Every call shares the array:
+ * calls that overlap on the GPU (unordered streams) race. Device-side status (timeouts, bounds) is
+ * cleared at the start of each call and is not reported by this entry point.
+ */
+CSA_API int csa_indexer_topk_noalloc(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
+                                     const uint16_t* q_idx, const float* w, const uint16_t* idx_cache,
+                                     int64_t idx_bstride, int max_entries, int32_t* topk_idx, void* stream);
+
+/*
  * csa_get_device_status -- synchronise `stream`, read the status word in `ws` into *status
  * (CSA_OK, CSA_ERR_TIMEOUT or CSA_ERR_BOUNDS) and clear it. Returns CSA_ERR_CUDA if the
  * stream itself reports an error.

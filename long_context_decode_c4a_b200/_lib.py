@@ -84,6 +84,8 @@ PROTOTYPES = {
     "csa_decode_fused": (c_int, [POINTER(DecodeArgs), c_void_p]),
     "hca_decode_fused": (c_int, [POINTER(HcaDecodeArgs), c_void_p]),
     "csa_get_device_status": (c_int, [c_void_p, c_void_p, POINTER(c_int)]),
+    "csa_indexer_topk_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_int64, c_int, c_void_p, c_void_p]),
 }
 
 _lib = None
