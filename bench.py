@@ -24,9 +24,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -74,52 +72,55 @@ def traffic_for(kernel: str, workload: str, files):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """SM clock and clock-event-reason samples taken through NVML (read-only queries) while the
+    timed steps run on the device: `poll_until(event)` samples every millisecond until the event
+    that closes the timed region has completed."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown", 0x8),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap", 0x4),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80))
 
     def __init__(self, device_index: int):
-        self.dev = device_index
-        self.proc = None
-        self.path = None
-
-    def start(self):
+        self.nv = None
+        self.handle = None
+        self.rows = []
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=self.out, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            try:
+                self.handle = nv.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+            except Exception:  # noqa: BLE001
+                self.handle = nv.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            self.nv = nv
+        except Exception:  # noqa: BLE001
+            self.nv = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
+    def sample(self):
+        if self.nv is None:
+            return
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.handle, self.nv.NVML_CLOCK_SM)
+            mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+            self.rows.append((mhz, mask))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def poll_until(self, event, period_s: float = 0.001):
+        while not event.query():
+            self.sample()
+            time.sleep(period_s)
+
+    def result(self):
+        if not self.rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        names = [n for n, attr, bit in self.REASONS
+                 if any(m & getattr(self.nv, attr, bit) for _, m in self.rows)]
+        return {"sm_mhz": statistics.median(r[0] for r in self.rows), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(names), "samples": len(self.rows), "source": "nvml"}
 
 
 def dist_setup(n_gpus: int):
@@ -225,14 +226,16 @@ def run_ours_decode(wl, args, world, rank):
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    clocks.start()
     t0.record()
     for k in range(args.steps):
         call(*sets[k % len(sets)], evs=stage_ev[k])
+        if k % 16 == 0:
+            clocks.sample()
     t1.record()
+    clocks.poll_until(t1)
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
+    clk = clocks.result()
     ms = t0.elapsed_time(t1) / args.steps
     ms = max_over_ranks(ms, world)
     for st, _ in sets:
@@ -314,8 +317,8 @@ def cpu_baseline_decode(wl, budget_s: float = 15.0):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="pro_csa_decode_32k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sets", type=int, default=4, help="rotating input sets")

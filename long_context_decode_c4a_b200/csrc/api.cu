@@ -171,6 +171,7 @@ CompressParams compress_params(const csa_compressor_cfg* c, int B, int S, const 
   p.rope_dim = c->rope_dim;
   p.rope_base = c->rope_base;
   p.eps = c->eps;
+  for (int i = 0; i < c->rope_dim / 2; ++i) p.inv_freq[i] = std::pow((double)c->rope_base, -2.0 * i / c->rope_dim);
   p.B = B;
   p.S = S;
   p.start_pos = start_pos;
@@ -183,7 +184,6 @@ CompressParams compress_params(const csa_compressor_cfg* c, int B, int S, const 
   p.cache_bstride = cache_bstride;
   p.max_entries = max_entries;
   p.cache_f32 = cache_f32;
-  p.fuse_state = S == 1 ? 1 : 0;
   p.status = status;
   return p;
 }
@@ -205,6 +205,11 @@ int check_compress_args(const csa_compressor_cfg* cfg, int B, int S, const int32
 }
 
 int launch_compress(const CompressLaunch& L, int nstreams, int B, int S, int ratio, cudaStream_t st) {
+  if (S == 1) {
+    compress_decode_kernel<<<dim3((unsigned)B, (unsigned)nstreams), kCompressThreads, 0, st>>>(L);
+    CSA_CUDA(cudaGetLastError());
+    return CSA_OK;
+  }
   const dim3 grid((unsigned)((S + ratio - 1) / ratio), (unsigned)B, (unsigned)nstreams);
   compress_kernel<<<grid, kCompressThreads, 0, st>>>(L);
   CSA_CUDA(cudaGetLastError());
@@ -391,7 +396,7 @@ int run_attn(const AttnArgs& a, bool csa_mode, cudaStream_t st) {
   P.H = a.H;
   P.d = a.d;
   P.rope_dim = a.rope_dim;
-  P.rope_base = a.rope_base;
+  for (int i = 0; i < a.rope_dim / 2; ++i) P.inv_freq[i] = std::pow((double)a.rope_base, -2.0 * i / a.rope_dim);
   P.scale_log2 = a.scale * 1.4426950408889634f;
   P.window = a.window;
   P.ring_cap = a.ring_cap;

@@ -25,6 +25,13 @@ namespace csa {
 
 namespace {
 
+// ReLU that keeps NaN (a NaN dot product stays NaN, as max(x, 0) does in IEEE propagation).
+__device__ __forceinline__ float relu_nan(float x) {
+  float r;
+  asm("max.NaN.f32 %0, %1, 0f00000000;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 struct ItemCoord {
   int b, qg, et;
 };
@@ -109,7 +116,7 @@ __device__ __forceinline__ void epilogue_tile(const IndexerParams& P, const floa
       for (int j = 0; j < 32; ++j) {
         const float x = __uint_as_float(v[j]);
         float& acc = part[j / kColsPerQ][j & 3];
-        acc = fmaf(w_s[col0 + 32 * c + j], fmaxf(x, 0.f), acc);
+        acc = fmaf(w_s[col0 + 32 * c + j], relu_nan(x), acc);
       }
     }
 #pragma unroll
@@ -171,6 +178,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  if (threadIdx.x == 0) trace_time(P.status, 599);
 
   const long long total = P.total_items;
   const long long per = (total + gridDim.x - 1) / gridDim.x;
@@ -205,6 +213,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         tma_load_2d(dst, &map_k, 0, krow, &sm.k_full[st]);
         tma_load_2d(dst + 16384, &map_k, 64, krow, &sm.k_full[st]);
         trace_mark(status, 0, (uint32_t)(100 + n));
+        if (n < 100) trace_time(status, 600 + (int)n);
         ++n;
       }
     }
@@ -241,6 +250,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         mma_commit(&sm.k_empty[st]);
         mma_commit(&sm.acc_full[a]);
         trace_mark(status, 1, (uint32_t)(100 + n));
+        if (n < 100) trace_time(status, 700 + (int)n);
         ++n;
       }
       // Every MMA issued by this thread completes before TMEM is released.
@@ -279,10 +289,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       const int a = (int)(my % n_acc);
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full[a], (uint32_t)((my / n_acc) & 1), abort_flag, status, 221))) break;
       if (gt == 0) trace_mark(status, 2, (uint32_t)(100 + my));
+      if (gt == 0 && my < 100) trace_time(status, 800 + (int)my);
       tc_fence_after();
       epilogue_tile<HI>(P, w_s, vis_s, tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(a * N), c.b, c.qg, c.et, row);
       tc_fence_before();
       mbar_arrive(&sm.acc_empty[a]);
+      if (gt == 0 && my < 100) trace_time(status, 900 + (int)my);
     }
   }
   __syncwarp();

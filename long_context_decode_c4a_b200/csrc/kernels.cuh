@@ -20,6 +20,7 @@ constexpr int kMaxKeepChunks = 4;
 struct CompressParams {
   int ratio, overlap, d, rope_dim;
   float rope_base, eps;
+  double inv_freq[kMaxRopePairs];   // rope_base^(-2i/rope_dim), formed on the host in double
   int B, S;
   const int32_t* start_pos;   // [B]
   const uint16_t* kv;         // [B, S, width]
@@ -31,8 +32,7 @@ struct CompressParams {
   long long cache_bstride;
   int max_entries;
   float* cache_f32;           // nullable, same layout as cache
-  int fuse_state;             // S == 1: the CTA of the (only) group slot also updates the state
-  // Window-ring write of the fused decode step (nullable win_src disables it).
+  // Window-ring write of the fused decode step (nullable win_src disables it; S == 1 only).
   const uint16_t* win_src;    // [B, d]
   uint16_t* ring;
   long long ring_bstride;
@@ -45,6 +45,7 @@ struct CompressLaunch {
 };
 
 __global__ void compress_kernel(CompressLaunch L);
+__global__ void compress_decode_kernel(CompressLaunch L);
 __global__ void compress_state_kernel(CompressLaunch L);
 __global__ void state_reset_kernel(uint16_t* kv, uint16_t* score, long long n);
 
@@ -98,7 +99,7 @@ __global__ void topk_merge_kernel(TopkParams P);
 
 // ------------------------------------------------------------------------------ attention (K4/K5)
 
-constexpr int kAttnThreads = 288;         // warps 0..3 gathers, warp 4 MMA, warps 5..8 softmax
+constexpr int kAttnThreads = 416;         // warps 0..3 gathers, warp 4 MMA, warps 5..12 softmax
 constexpr int kAttnMaxWindow = 1024;
 constexpr int kAttnMaxTopk = 2048;
 constexpr int kAttnMaxCompressed = 2048;  // HCA: visible entries read per query
@@ -107,7 +108,8 @@ constexpr int kAttnMaxTiles = kAttnMaxCands / 64;
 
 struct AttnParams {
   int B, S, H, d, rope_dim;
-  float rope_base, scale_log2;            // scale * log2(e)
+  float scale_log2;                       // scale * log2(e)
+  double inv_freq[kMaxRopePairs];         // rope_base^(-2i/rope_dim), formed on the host in double
   int window, ring_cap;
   long long ring_rows;                    // ring rows per request (ring_bstride / d)
   long long cache_rows;                   // cache rows per request (cache_bstride / d)

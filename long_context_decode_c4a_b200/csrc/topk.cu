@@ -5,13 +5,15 @@
 // indices of <= topK compressed entries. Ties go to the lower index; the output lists the chosen
 // indices in ascending order, padded with -1.
 //
-// Method: block-level radix select on order-preserving 32-bit keys (8 bits per pass, MSB first)
-// finds the k-th largest key T and how many keys equal to T to keep; a compaction pass in index
-// order then keeps every key > T and the first `need` keys == T. Inputs of up to kSmemKeys
-// entries are staged once in shared memory; longer score rows are cut into chunks whose local
-// top-k lists (in index order) are merged by a second launch with the same routine. The global
-// order (score desc, index asc) restricted to a chunk is the chunk's own order, so the global
-// top-k is contained in the union of the chunks' top-k lists.
+// Method: block-level radix select on order-preserving 32-bit keys finds the k-th largest key T
+// and how many keys equal to T to keep; a compaction pass in index order then keeps every key > T
+// and the first `need` keys == T. Each radix pass bins the keys of the current key range into at
+// most 2048 equal bins (the first range is [min, max] of the keys, so the bins follow the data's
+// own spread and the shared-memory counters see little contention); three passes always suffice.
+// A chunk of up to 16384 scores is held in registers (16 per thread); longer score rows are cut
+// into chunks whose local top-k lists (in index order) are merged by a second launch with the
+// same routine. The global order (score desc, index asc) restricted to a chunk is the chunk's own
+// order, so the global top-k is contained in the union of the chunks' top-k lists.
 
 #include "kernels.cuh"
 
@@ -19,18 +21,117 @@ namespace csa {
 
 namespace {
 
-// Order-preserving key: larger score -> larger key; -0 == +0; NaN below every number.
+// Order-preserving key, offset by one so that 0 can mark an empty position: larger score ->
+// larger key; -0 == +0; NaN (key 1) below every number; +inf -> 0xFF800001.
 __device__ __forceinline__ uint32_t score_key(float f) {
-  if (f != f) return 0u;
+  if (f != f) return 1u;
   uint32_t u = __float_as_uint(f);
   if (u == 0x80000000u) u = 0u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((u & 0x80000000u) ? ~u : (u | 0x80000000u)) + 1u;
+}
+
+constexpr int kSelBits = 11;
+constexpr int kSelBins = 1 << kSelBits;   // histogram bins per pass (2 per thread at 1024 threads)
+
+struct SelectShared {
+  uint32_t hist[kSelBins];
+  uint32_t wred[32][3];
+  uint32_t bin, above;
+};
+
+// The k-th largest key T among the nonzero keys of the block, and how many keys equal to T the
+// top k holds (need = k - #keys > T). take_all: at most k nonzero keys, all of them are chosen.
+struct Threshold {
+  uint32_t T, need;
+  bool take_all;
+};
+
+// Radix select over an adaptive key range. The range starts as [min, max] of the keys; each pass
+// splits the current range into at most kSelBins equal power-of-two bins, counts the keys of the
+// range per bin, and narrows the range to the bin that holds the krem-th largest key. A range of
+// up to 2^32 keys needs at most three passes (bin widths <= 2^21, <= 2^10, 1). `each(f)` calls
+// f(key) for every key the calling thread owns; all threads of the block must call this.
+template <class ForEach>
+__device__ Threshold select_threshold(int k, ForEach each, SelectShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  uint32_t c = 0, mn = 0xFFFFFFFFu, mx = 0u;
+  each([&](uint32_t key) {
+    if (key != 0u) {
+      ++c;
+      mn = min(mn, key);
+      mx = max(mx, key);
+    }
+  });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    sh.wred[w][0] = c;
+    sh.wred[w][1] = mn;
+    sh.wred[w][2] = mx;
+  }
+  __syncthreads();
+  uint32_t total = 0, lo = 0xFFFFFFFFu, hi = 0u;
+  for (int i = 0; i < nw; ++i) {
+    total += sh.wred[i][0];
+    lo = min(lo, sh.wred[i][1]);
+    hi = max(hi, sh.wred[i][2]);
+  }
+  Threshold r;
+  if (total <= (uint32_t)k) {
+    r.take_all = true;
+    r.T = 1u;
+    r.need = 0u;
+    return r;
+  }
+  uint32_t krem = (uint32_t)k;  // rank of T counted from the top of [lo, hi]
+  while (lo != hi) {
+    const uint32_t range = hi - lo;
+    const int shift = range < (uint32_t)kSelBins ? 0 : (32 - __clz((int)range)) - kSelBits;
+    const int nb = (int)(range >> shift) + 1;
+    for (int i = tid; i < nb; i += blockDim.x) sh.hist[i] = 0u;
+    __syncthreads();
+    each([&](uint32_t key) {
+      if (key >= lo && key <= hi) atomicAdd(&sh.hist[(key - lo) >> shift], 1u);
+    });
+    __syncthreads();
+    // Thread t owns bins nb-1-2t and nb-2-2t: a scan in thread order runs over descending bins.
+    const int b0 = nb - 1 - 2 * tid, b1 = b0 - 1;
+    const uint32_t h0 = b0 >= 0 ? sh.hist[b0] : 0u, h1 = b1 >= 0 ? sh.hist[b1] : 0u;
+    const uint32_t s = h0 + h1;
+    uint32_t incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) sh.wred[w][0] = incl;
+    __syncthreads();
+    uint32_t excl = incl - s;
+    for (int i = 0; i < w; ++i) excl += sh.wred[i][0];
+    if (excl < krem && excl + s >= krem) {
+      const bool first = excl + h0 >= krem;
+      sh.bin = (uint32_t)(first ? b0 : b1);
+      sh.above = first ? excl : excl + h0;
+    }
+    __syncthreads();
+    krem -= sh.above;
+    const uint32_t nlo = lo + (sh.bin << shift);
+    hi = min(hi, nlo + ((1u << shift) - 1u));
+    lo = nlo;
+  }
+  r.take_all = false;
+  r.T = lo;
+  r.need = krem;
+  return r;
 }
 
 struct TopkShared {
-  uint32_t hist[256];
+  SelectShared sel;
   uint32_t warp_tot[32][2];
-  uint32_t digit, above, total;
 };
 
 // Exclusive prefix of two per-thread counts across the block (thread order), and the totals.
@@ -69,194 +170,72 @@ __device__ __forceinline__ void block_scan2(uint32_t a, uint32_t b, TopkShared& 
   tot_b = tb;
 }
 
-// Select the top k of n keys (key(i), valid(i)) with ties to the lower position, and call
-// emit(pos, i) for the chosen positions in increasing i (pos = 0, 1, ...). Returns the count.
-// Each thread owns the contiguous positions [tid*per, tid*per + per).
+// Select the top k of the n keys key_of(i) (0 = empty position) with ties to the lower position,
+// and call emit(pos, i) for the chosen positions in increasing i (pos = 0, 1, ...). Returns the
+// count. Each thread owns the contiguous positions [tid*per, tid*per + per); keys are re-read on
+// every pass, so key_of should read memory that stays in cache.
 template <class KeyFn, class EmitFn>
 __device__ uint32_t block_topk(int n, int k, KeyFn key_of, EmitFn emit, TopkShared& sh) {
   const int tid = threadIdx.x;
   const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
   const int lo = min(n, tid * per), hi = min(n, lo + per);
-  // Count valid entries.
-  uint32_t cnt = 0;
-  for (int i = lo; i < hi; ++i) {
-    bool v;
-    (void)key_of(i, v);
-    cnt += v ? 1u : 0u;
-  }
-  {
-    uint32_t pa, pb, ta, tb;
-    block_scan2(cnt, 0u, sh, pa, pb, ta, tb);
-    cnt = ta;
-  }
-  const bool take_all = (int)cnt <= k;
-  uint32_t prefix = 0, mask = 0;
-  int krem = k;
-  if (!take_all) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += blockDim.x) sh.hist[i] = 0;
-      __syncthreads();
-      // Warp-aggregated histogram: lanes holding the same digit add once.
-      for (int r = 0; r < per; ++r) {
-        const int i = lo + r;
-        bool v = false;
-        uint32_t key = 0;
-        if (i < hi) key = key_of(i, v);
-        const bool live = v && (key & mask) == prefix;
-        const uint32_t dig = live ? ((key >> shift) & 255u) : 256u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, dig);
-        if (live && (__ffs(peers) - 1) == (int)(threadIdx.x & 31)) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
-      }
-      __syncthreads();
-      if (tid < 32) {
-        // lane L owns bins 255-8L .. 248-8L (descending); find the bin where the count of keys
-        // with a larger digit first reaches krem.
-        uint32_t loc[8];
-        uint32_t s = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          loc[j] = sh.hist[255 - 8 * tid - j];
-          s += loc[j];
-        }
-        uint32_t incl = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += y;
-        }
-        const uint32_t excl = incl - s;
-        if (excl < (uint32_t)krem && incl >= (uint32_t)krem) {
-          uint32_t run = excl;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (run + loc[j] >= (uint32_t)krem) {
-              sh.digit = 255 - 8 * tid - j;
-              sh.above = run;
-              break;
-            }
-            run += loc[j];
-          }
-        }
-      }
-      __syncthreads();
-      krem -= (int)sh.above;
-      prefix |= sh.digit << shift;
-      mask |= 0xFFu << shift;
-    }
-  }
+  const Threshold th = select_threshold(k, [&](auto&& f) {
+    for (int i = lo; i < hi; ++i) f(key_of(i));
+  }, sh.sel);
   // Compaction in index order: keep every key > T and the first `need` keys == T.
-  const uint32_t T = prefix;
-  const uint32_t need = take_all ? 0u : (uint32_t)krem;
   uint32_t n_gt = 0, n_eq = 0;
   for (int i = lo; i < hi; ++i) {
-    bool v;
-    const uint32_t key = key_of(i, v);
-    if (!v) continue;
-    if (take_all || key > T) ++n_gt;
-    else if (key == T) ++n_eq;
+    const uint32_t key = key_of(i);
+    if (key == 0u) continue;
+    if (th.take_all || key > th.T) ++n_gt;
+    else if (key == th.T) ++n_eq;
   }
   uint32_t pre_gt, pre_eq, tot_gt, tot_eq;
   block_scan2(n_gt, n_eq, sh, pre_gt, pre_eq, tot_gt, tot_eq);
   uint32_t eq_seen = pre_eq;                            // keys == T before this thread's range
-  uint32_t pos = pre_gt + min(pre_eq, need);            // output slot of the next selected key
+  uint32_t pos = pre_gt + min(pre_eq, th.need);         // output slot of the next selected key
   for (int i = lo; i < hi; ++i) {
-    bool v;
-    const uint32_t key = key_of(i, v);
-    if (!v) continue;
-    if (take_all || key > T) {
+    const uint32_t key = key_of(i);
+    if (key == 0u) continue;
+    if (th.take_all || key > th.T) {
       emit(pos++, i);
-    } else if (key == T) {
-      if (eq_seen < need) emit(pos++, i);
+    } else if (key == th.T) {
+      if (eq_seen < th.need) emit(pos++, i);
       ++eq_seen;
     }
   }
-  return tot_gt + min(tot_eq, need);
+  return tot_gt + min(tot_eq, th.need);
 }
 
 constexpr int kRegKeys = kTopkChunk / kTopkThreads;   // keys per thread in the chunk kernel (16)
 
 struct TopkRegShared {
-  uint32_t hist[256];
+  SelectShared sel;
   uint32_t cnt[kRegKeys][32][2];   // per (key slot, warp): count of keys > T, == T
   uint32_t off[kRegKeys][32][2];   // exclusive prefix over warps
   uint32_t base[kRegKeys][2];      // keys > T / == T in all earlier key slots
-  uint32_t red[32];
-  uint32_t digit, above, total;
+  uint32_t above, total;
 };
 
-// Top-k of up to kRegKeys * blockDim keys held in registers. Thread t holds the keys of positions
-// i = r * blockDim + t (r = 0 .. kRegKeys-1). Chosen positions are passed to emit(pos, r) with
-// pos = 0, 1, ... in increasing i. Returns the count.
+// Top-k of up to kRegKeys * blockDim keys held in registers (0 = empty position). Thread t holds
+// the keys of positions i = r * blockDim + t (r = 0 .. kRegKeys-1). Chosen positions are passed to
+// emit(pos, r) with pos = 0, 1, ... in increasing i. Returns the count.
 template <class EmitFn>
-__device__ uint32_t block_topk_regs(const uint32_t (&key)[kRegKeys], int n, int k, EmitFn emit, TopkRegShared& sh) {
+__device__ uint32_t block_topk_regs(const uint32_t (&key)[kRegKeys], int k, EmitFn emit, TopkRegShared& sh) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
-  auto valid = [&](int r) { return r * (int)blockDim.x + tid < n; };
-  uint32_t cnt = 0;
+  const Threshold th = select_threshold(k, [&](auto&& f) {
 #pragma unroll
-  for (int r = 0; r < kRegKeys; ++r) cnt += valid(r) ? 1u : 0u;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) sh.red[w] = cnt;
-  __syncthreads();
-  uint32_t total = 0;
-  for (int i = 0; i < nw; ++i) total += sh.red[i];
-  const bool take_all = (int)total <= k;
-  uint32_t prefix = 0, mask = 0;
-  int krem = k;
-  if (!take_all) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = tid; i < 256; i += blockDim.x) sh.hist[i] = 0;
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < kRegKeys; ++r) {
-        const bool live = valid(r) && (key[r] & mask) == prefix;
-        const uint32_t dig = live ? ((key[r] >> shift) & 255u) : 256u;
-        const uint32_t peers = __match_any_sync(0xffffffffu, dig);
-        if (live && (__ffs(peers) - 1) == lane) atomicAdd(&sh.hist[dig], (uint32_t)__popc(peers));
-      }
-      __syncthreads();
-      if (tid < 32) {
-        uint32_t loc[8];
-        uint32_t s = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          loc[j] = sh.hist[255 - 8 * tid - j];
-          s += loc[j];
-        }
-        uint32_t incl = s;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (tid >= o) incl += y;
-        }
-        const uint32_t excl = incl - s;
-        if (excl < (uint32_t)krem && incl >= (uint32_t)krem) {
-          uint32_t run = excl;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (run + loc[j] >= (uint32_t)krem) {
-              sh.digit = 255 - 8 * tid - j;
-              sh.above = run;
-              break;
-            }
-            run += loc[j];
-          }
-        }
-      }
-      __syncthreads();
-      krem -= (int)sh.above;
-      prefix |= sh.digit << shift;
-      mask |= 0xFFu << shift;
-    }
-  }
+    for (int r = 0; r < kRegKeys; ++r) f(key[r]);
+  }, sh.sel);
   // Compaction in index order: keep every key > T and the first `need` keys == T.
-  const uint32_t T = prefix;
-  const uint32_t need = take_all ? 0u : (uint32_t)krem;
+  const uint32_t T = th.T;
+  const uint32_t need = th.need;
+  const bool take_all = th.take_all;
   const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
   for (int r = 0; r < kRegKeys; ++r) {
-    const bool gt = valid(r) && (take_all || key[r] > T);
-    const bool eq = valid(r) && !take_all && key[r] == T;
+    const bool gt = take_all ? key[r] != 0u : key[r] > T;
+    const bool eq = !take_all && key[r] == T;
     const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
     const uint32_t beq = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) {
@@ -297,8 +276,8 @@ __device__ uint32_t block_topk_regs(const uint32_t (&key)[kRegKeys], int n, int 
   __syncthreads();
 #pragma unroll
   for (int r = 0; r < kRegKeys; ++r) {
-    const bool gt = valid(r) && (take_all || key[r] > T);
-    const bool eq = valid(r) && !take_all && key[r] == T;
+    const bool gt = take_all ? key[r] != 0u : key[r] > T;
+    const bool eq = !take_all && key[r] == T;
     const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
     const uint32_t beq = __ballot_sync(0xffffffffu, eq);
     if (!(gt || eq)) continue;
@@ -348,7 +327,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
     key[r] = i < n ? score_key(row[i]) : 0u;
   }
   if (nchunks <= 1) {
-    const uint32_t cnt = block_topk_regs(key, n, P.topk, [&](uint32_t pos, int r) {
+    const uint32_t cnt = block_topk_regs(key, P.topk, [&](uint32_t pos, int r) {
       out[pos] = lo + r * (int)blockDim.x + (int)threadIdx.x;
     }, sh);
     for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
@@ -356,7 +335,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
     const long long cb = ((long long)q * P.max_chunks + c) * P.topk;
     uint32_t* ck = P.cand_key + cb;
     int32_t* ci = P.cand_idx + cb;
-    const uint32_t cnt = block_topk_regs(key, n, P.topk, [&](uint32_t pos, int r) {
+    const uint32_t cnt = block_topk_regs(key, P.topk, [&](uint32_t pos, int r) {
       ck[pos] = key[r];
       ci[pos] = lo + r * (int)blockDim.x + (int)threadIdx.x;
     }, sh);
@@ -384,10 +363,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) 
   const int32_t* ci = P.cand_idx + cb;
   const int n = nchunks * P.topk;
   const int K = P.topk;
-  auto key_of = [&](int i, bool& v) -> uint32_t {
-    v = (i % K) < cnts[i / K];
-    return v ? ck[i] : 0u;
-  };
+  auto key_of = [&](int i) -> uint32_t { return (i % K) < cnts[i / K] ? ck[i] : 0u; };
   int32_t* out = P.out + (long long)q * P.topk;
   const uint32_t cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = ci[i]; }, sh);
   for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;

@@ -93,3 +93,41 @@ def test_topk_edge_cases(ops):
     assert np.all(idx[0, 0] == -1) and np.all(idx[0, 1] == -1)
     assert np.array_equal(idx[0, 2], np.r_[np.arange(10), -np.ones(6)])
     assert np.array_equal(idx[0, 3], np.arange(16))
+
+
+@pytest.mark.parametrize("case", ["all_equal", "one_outlier", "inf_nan", "wide_range", "two_values"])
+def test_topk_adversarial_score_distributions(ops, case):
+    """Score rows whose shape stresses the radix select: one value everywhere, a single far
+    outlier above a tie, +-inf and NaN scores (NaN ranks last), scores spread over ~2^100, and two
+    distinct values. The selection must equal the oracle's order on the very scores the GPU wrote."""
+    B, S, H_I, topk = 2, 1, 64, 1024
+    E = 6000 if case != "wide_range" else 16000
+    q_idx, w, cache = _inputs(B, S, H_I, E, seed=17)
+    if case == "all_equal":
+        cache[:] = cache[:, :1]
+    elif case == "one_outlier":
+        cache[:] = cache[:, :1]
+        cache[:, 4321] = cache[:, 4321] * 64
+    elif case == "inf_nan":
+        # q dims 5 and 9 > 0; request 0 weights all < 0, request 1 all > 0: a row with +inf in
+        # dim 5 scores -inf (request 0) or +inf (request 1); +inf in 5 with -inf in 9 gives NaN.
+        q_idx[..., 5] = q_idx[..., 5].abs() + 0.1
+        q_idx[..., 9] = q_idx[..., 9].abs() + 0.1
+        w[0] = -w[0].abs()
+        w[1] = w[1].abs()
+        cache[:, ::97, 5] = float("inf")
+        cache[:, 3::89, 5] = float("inf")
+        cache[:, 3::89, 9] = -float("inf")
+    elif case == "wide_range":
+        scale = torch.exp2(torch.randint(-50, 50, (B, E, 1)).float())
+        cache = (cache.float() * scale).to(torch.bfloat16)
+    elif case == "two_values":
+        cache[:] = cache[:, :1]
+        cache[:, 1::3] = cache[:, 1::3] * 2
+    pos = torch.full((B, S), 4 * E - 1, dtype=torch.int32)
+    sc, idx = _run(ops, pos, q_idx, w, cache, topk)
+    if case == "inf_nan":
+        assert np.isnan(sc[:, 0, :E]).all(axis=0).any()
+        assert (sc[0, 0, :E] == -np.inf).any() and (sc[1, 0, :E] == np.inf).any()
+    for b in range(B):
+        assert np.array_equal(idx[b, 0], O.topk_select(sc[b, 0, :E], topk)), f"b={b}"
