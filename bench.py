@@ -206,30 +206,56 @@ def run_ours_decode(wl, args, world, rank):
         del inp
     torch.cuda.synchronize()
 
-    def call(st, x, evs=None):
+    preps = []
+    for st, x in sets:
         if csa:
-            st.step(x["pos"], x["kv"], x["score"], x["idx_kv"], x["idx_score"], x["win_kv"], x["q"], x["q_idx"],
-                    x["w"], x["sink"], out=x["out"], stage_events=evs)
+            preps.append(st.prepare(x["pos"], x["kv"], x["score"], x["idx_kv"], x["idx_score"], x["win_kv"], x["q"],
+                                    x["q_idx"], x["w"], x["sink"], out=x["out"]))
         else:
-            st.step(x["pos"], x["kv"], x["score"], x["win_kv"], x["q"], x["sink"], out=x["out"], stage_events=evs)
+            preps.append(st.prepare(x["pos"], x["kv"], x["score"], x["win_kv"], x["q"], x["sink"], out=x["out"]))
+
+    def call(i, evs=None):
+        preps[i % len(preps)].launch(stage_events=evs)
 
     nstage = 5 if csa else 3
     for i in range(args.warmup):
-        call(*sets[i % len(sets)])
+        call(i)
     torch.cuda.synchronize()
-    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
-    for row in stage_ev:       # create the underlying events before the timed region
-        for e in row:
-            e.record()
+    # One CUDA graph holds one step of every input set (the launches keep their programmatic
+    # dependencies); the timed region replays it and launches any remaining steps directly.
+    graph = None
+    if args.graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for i in range(len(preps)):
+                call(i)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for i in range(len(preps)):
+                call(i)
+        torch.cuda.synchronize()
+        for _ in range(max(1, args.warmup // len(preps))):
+            graph.replay()
+        torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(torch.cuda.current_device())
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     t0.record()
-    for k in range(args.steps):
-        call(*sets[k % len(sets)], evs=stage_ev[k])
-        if k % 16 == 0:
+    k = 0
+    if graph is not None:
+        while k + len(preps) <= args.steps:
+            graph.replay()
+            k += len(preps)
+            if (k // len(preps)) % 4 == 0:
+                clocks.sample()
+    for kk in range(k, args.steps):
+        call(kk)
+        if kk % 16 == 0:
             clocks.sample()
     t1.record()
     clocks.poll_until(t1)
@@ -238,11 +264,23 @@ def run_ours_decode(wl, args, world, rank):
     clk = clocks.result()
     ms = t0.elapsed_time(t1) / args.steps
     ms = max_over_ranks(ms, world)
+    del graph
     for st, _ in sets:
         status = ops.device_status(st.ws)
         if status != 0:
             raise RuntimeError(f"device status {status} after the timed steps")
 
+    # ---- per-kernel durations: the same steps again with CUDA events recorded between the kernels
+    # on the launching stream (an event between two kernels also ends their launch overlap, so
+    # these steps run separately from the timed ones above)
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
+    for row in stage_ev:       # create the underlying events before the loop
+        for e in row:
+            e.record()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        call(k, evs=stage_ev[k])
+    torch.cuda.synchronize()
     stage_names = ["compress", "indexer", "topk", "attention"] if csa else ["compress", "attention"]
     stage_ms = {n: statistics.mean(stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(args.steps))
                 for i, n in enumerate(stage_names)}
@@ -255,14 +293,23 @@ def run_ours_decode(wl, args, world, rank):
     d2h = out_host.numel() * out_host.element_size()
     dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
 
-    def e2e_step(i):
-        stt, xx = sets[i % len(sets)]
-        for k, v in host.items():
-            dev_in[k].copy_(v, non_blocking=True)
+    e2e_preps = []
+    for stt, xx in sets:
         xin = dict(xx)
         xin.update(dev_in)
-        call(stt, xin)
-        out_host.copy_(xin["out"], non_blocking=True)
+        if csa:
+            e2e_preps.append(stt.prepare(xin["pos"], xin["kv"], xin["score"], xin["idx_kv"], xin["idx_score"],
+                                         xin["win_kv"], xin["q"], xin["q_idx"], xin["w"], xin["sink"],
+                                         out=xin["out"]))
+        else:
+            e2e_preps.append(stt.prepare(xin["pos"], xin["kv"], xin["score"], xin["win_kv"], xin["q"], xin["sink"],
+                                         out=xin["out"]))
+
+    def e2e_step(i):
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        out = e2e_preps[i % len(e2e_preps)].launch()
+        out_host.copy_(out, non_blocking=True)
 
     for i in range(args.warmup):
         e2e_step(i)
@@ -324,6 +371,8 @@ def main(argv=None):
     ap.add_argument("--sets", type=int, default=4, help="rotating input sets")
     ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch every timed step from the host instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -366,7 +415,9 @@ def main(argv=None):
                    "compressed_entries": wl.max_entries, "window": wl.W, "heads": wl.H, "head_dim": wl.d,
                    "indexer_heads": wl.H_I, "topk": wl.topk, "reads_per_query": reads,
                    "parallelism": f"requests sharded over {world} GPU(s), no data-path collective",
-                   "l2": f"{args.sets} rotating input sets, each step reads {total_bytes / 1e6:.0f} MB > 126 MB L2"},
+                   "l2": f"{args.sets} rotating input sets, each step reads {total_bytes / 1e6:.0f} MB > 126 MB L2",
+                   "launch": ("CUDA graph of one step per input set, replayed" if args.graph
+                              else "every step launched from the host")},
         "tokens_per_s": value,
         "step_hbm_gbs": total_bytes / (r["ms"] * 1e-3) / 1e9,
         "step_hbm_frac": total_bytes / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],

@@ -13,6 +13,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "csa.h"
 #include "kernels.cuh"
@@ -89,6 +90,24 @@ struct DeviceInfo {
   int max_smem = 0;
   bool attrs_set = false;
 };
+
+// Launch with programmatic stream serialization: the kernel may begin launching while the
+// previous kernel on the stream runs; it calls pdl_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 int device_info(DeviceInfo** out) {
   static DeviceInfo info[64];
@@ -206,16 +225,13 @@ int check_compress_args(const csa_compressor_cfg* cfg, int B, int S, const int32
 
 int launch_compress(const CompressLaunch& L, int nstreams, int B, int S, int ratio, cudaStream_t st) {
   if (S == 1) {
-    compress_decode_kernel<<<dim3((unsigned)B, (unsigned)nstreams), kCompressThreads, 0, st>>>(L);
-    CSA_CUDA(cudaGetLastError());
+    CSA_CUDA(launch_pdl(compress_decode_kernel, dim3((unsigned)B, (unsigned)nstreams), dim3(kCompressThreads), 0, st, L));
     return CSA_OK;
   }
   const dim3 grid((unsigned)((S + ratio - 1) / ratio), (unsigned)B, (unsigned)nstreams);
-  compress_kernel<<<grid, kCompressThreads, 0, st>>>(L);
-  CSA_CUDA(cudaGetLastError());
+  CSA_CUDA(launch_pdl(compress_kernel, grid, dim3(kCompressThreads), 0, st, L));
   if (S > 1) {
-    compress_state_kernel<<<dim3((unsigned)B, 1, (unsigned)nstreams), kCompressThreads, 0, st>>>(L);
-    CSA_CUDA(cudaGetLastError());
+    CSA_CUDA(launch_pdl(compress_state_kernel, dim3((unsigned)B, 1, (unsigned)nstreams), dim3(kCompressThreads), 0, st, L));
   }
   return CSA_OK;
 }
@@ -296,16 +312,17 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
   if (int rc = make_map_2d(&map_k, a.idx_cache, 128, (uint64_t)a.B * P.rows_per_req, 128, 64, 128)) return rc;
   if (int rc = make_map_2d(&map_q, a.q_idx, 128, (uint64_t)queries * a.H_I, 128, 64, (uint32_t)P.N)) return rc;
   const size_t smem = indexer_smem_bytes(stages, P.N);
-  const unsigned grid = (unsigned)std::min<long long>(P.total_items, dev->sms);
+  const dim3 grid((unsigned)std::min<long long>(P.total_items, dev->sms));
+  cudaError_t e = cudaSuccess;
   switch (a.H_I) {
-    case 4: indexer_kernel<4><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
-    case 8: indexer_kernel<8><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
-    case 16: indexer_kernel<16><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
-    case 32: indexer_kernel<32><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
-    case 64: indexer_kernel<64><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
-    default: indexer_kernel<128><<<grid, kIdxThreads, smem, st>>>(map_k, map_q, P); break;
+    case 4: e = launch_pdl(indexer_kernel<4>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+    case 8: e = launch_pdl(indexer_kernel<8>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+    case 16: e = launch_pdl(indexer_kernel<16>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+    case 32: e = launch_pdl(indexer_kernel<32>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+    case 64: e = launch_pdl(indexer_kernel<64>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+    default: e = launch_pdl(indexer_kernel<128>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
   }
-  CSA_CUDA(cudaGetLastError());
+  CSA_CUDA(e);
   if (ev) CSA_CUDA(cudaEventRecord(ev[0], st));
 
   TopkParams T{};
@@ -323,12 +340,10 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
   T.cand_cnt = reinterpret_cast<int*>(ws + L.cand_cnt_off);
   T.status = status;
   const int nchunks = std::max(1, L.max_chunks);
-  topk_chunk_kernel<<<dim3((unsigned)nchunks, (unsigned)queries), kTopkThreads, 0, st>>>(T);
-  CSA_CUDA(cudaGetLastError());
+  CSA_CUDA(launch_pdl(topk_chunk_kernel, dim3((unsigned)nchunks, (unsigned)queries), dim3(kTopkThreads), 0, st, T));
   if (L.max_chunks > 1) {
     CSA_CHECK_SUP(L.max_chunks <= kTopkMaxChunks, "max_entries too large for the top-k merge");
-    topk_merge_kernel<<<(unsigned)queries, kTopkThreads, 0, st>>>(T);
-    CSA_CUDA(cudaGetLastError());
+    CSA_CUDA(launch_pdl(topk_merge_kernel, dim3((unsigned)queries), dim3(kTopkThreads), 0, st, T));
   }
   if (ev) CSA_CUDA(cudaEventRecord(ev[1], st));
   return CSA_OK;
@@ -419,8 +434,7 @@ int run_attn(const AttnArgs& a, bool csa_mode, cudaStream_t st) {
   const size_t smem = attn_smem_bytes();
   CSA_CHECK_SUP(smem <= (size_t)dev->max_smem, "shared memory too small for the attention kernel");
   CSA_CHECK_SUP(queries <= 65535, "at most 65535 queries per call");
-  attn_kernel<<<dim3(2, (unsigned)queries), kAttnThreads, smem, st>>>(map_q, P);
-  CSA_CUDA(cudaGetLastError());
+  CSA_CUDA(launch_pdl(attn_kernel, dim3(2, (unsigned)queries), dim3(kAttnThreads), smem, st, map_q, P));
   return CSA_OK;
 }
 

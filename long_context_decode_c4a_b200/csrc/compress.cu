@@ -153,6 +153,8 @@ __device__ void update_state(const CompressParams& P, int b, long long start, lo
 // Segments of S > 1 tokens (prefill): grid (group slots, B, streams); block kCompressThreads.
 // compress_state_kernel then brings the state to the end of the segment.
 __global__ void __launch_bounds__(kCompressThreads) compress_kernel(CompressLaunch L) {
+  pdl_wait();
+  pdl_trigger();
   const CompressParams& P = L.p[blockIdx.z];
   const int b = blockIdx.y;
   if (b >= P.B) return;
@@ -317,23 +319,14 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
   const int c = tid % C, grp = tid / C;
   const int c0 = c * 8;
   const int t = P.start_pos[b];
-  if (t < 0) {
-    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
-    return;
-  }
-  const int g = t / RATIO;
-  const int cur = kOverlap ? RATIO + t % RATIO : t % RATIO;  // state row of token t
-  const bool done = (t + 1) % RATIO == 0;
   uint16_t* skv = P.state_kv + (size_t)b * kRows * kWidth;
   uint16_t* ssc = P.state_score + (size_t)b * kRows * kWidth;
   const uint16_t* xkv = P.kv + (size_t)b * kWidth;  // token t's row (S == 1)
   const uint16_t* xsc = P.score + (size_t)b * kWidth;
-
-  // Window-ring write of the fused decode step.
-  if (P.win_src != nullptr && tid < D / 8) {
-    uint16_t* dst = P.ring + (long long)b * P.ring_bstride + (long long)(t % P.ring_cap) * D;
-    *reinterpret_cast<uint4*>(dst + c0) = *reinterpret_cast<const uint4*>(P.win_src + (size_t)b * D + c0);
-  }
+  // C4A reads its state rows before t is known: if t completes a group, token t is the last cur
+  // row (row 2*RATIO-1), so every slot and roll source is fixed; when t does not complete a group
+  // the values read are not used. C128A reads its (many) rows only for completing tokens.
+  constexpr int kLastRow = kRows - 1;
   // Token t's row, written to state row `cur` after the barrier.
   uint4 tok_kv = make_uint4(0, 0, 0, 0), tok_sc = make_uint4(0, 0, 0, 0);
   if (tid < kRowChunks) {
@@ -342,18 +335,31 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
   }
   // C4A roll: after group g completes, pre rows <- cur rows (token t's row from the input).
   uint4 roll_kv[kRollPer > 0 ? kRollPer : 1], roll_sc[kRollPer > 0 ? kRollPer : 1];
-  if (kOverlap && done) {
+  if (kOverlap) {
 #pragma unroll
     for (int k = 0; k < kRollPer; ++k) {
       const int idx = tid + k * kCompressThreads;
       if (idx < kRollChunks) {
         const int row = RATIO + idx / kRowChunks, ch = idx % kRowChunks;
-        const uint16_t* sk = row == cur ? xkv : skv + (size_t)row * kWidth;
-        const uint16_t* ss = row == cur ? xsc : ssc + (size_t)row * kWidth;
+        const uint16_t* sk = row == kLastRow ? xkv : skv + (size_t)row * kWidth;
+        const uint16_t* ss = row == kLastRow ? xsc : ssc + (size_t)row * kWidth;
         roll_kv[k] = *reinterpret_cast<const uint4*>(sk + ch * 8);
         roll_sc[k] = *reinterpret_cast<const uint4*>(ss + ch * 8);
       }
     }
+  }
+  if (t < 0) {
+    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    return;
+  }
+  const int g = t / RATIO;
+  const int cur = kOverlap ? RATIO + t % RATIO : t % RATIO;  // state row of token t
+  const bool done = (t + 1) % RATIO == 0;
+
+  // Window-ring write of the fused decode step.
+  if (P.win_src != nullptr && tid < D / 8) {
+    uint16_t* dst = P.ring + (long long)b * P.ring_bstride + (long long)(t % P.ring_cap) * D;
+    *reinterpret_cast<uint4*>(dst + c0) = *reinterpret_cast<const uint4*>(P.win_src + (size_t)b * D + c0);
   }
   // Partial softmax over this thread's slots, in the log2 domain.
   DecodePartial pt;
@@ -363,7 +369,7 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
     pt.s[i] = 0.f;
     pt.a[i] = 0.f;
   }
-  if (done) {
+  if (kOverlap || done) {
 #pragma unroll 1
     for (int k0 = 0; k0 < kPer; k0 += kBatch) {
       uint4 kraw[kBatch], sraw[kBatch];
@@ -376,14 +382,13 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
         if (kOverlap) {
           row = j;                              // pre rows 0..RATIO-1 (channels [0, D)), cur rows after
           coff = j < RATIO ? c0 : D + c0;
-          if (j < RATIO && g == 0) have[u] = false;  // no group before group 0: weight 0
         } else {
           row = j;
           coff = c0;
         }
         if (have[u]) {
-          const uint16_t* sk = row == cur ? xkv : skv + (size_t)row * kWidth;
-          const uint16_t* ss = row == cur ? xsc : ssc + (size_t)row * kWidth;
+          const uint16_t* sk = row == kLastRow ? xkv : skv + (size_t)row * kWidth;  // done: cur == kLastRow
+          const uint16_t* ss = row == kLastRow ? xsc : ssc + (size_t)row * kWidth;
           kraw[u] = *reinterpret_cast<const uint4*>(sk + coff);
           sraw[u] = *reinterpret_cast<const uint4*>(ss + coff);
         }
@@ -391,6 +396,7 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         if (!have[u]) continue;
+        if (kOverlap && grp + (k0 + u) * G < RATIO && g == 0) continue;  // no group before group 0: weight 0
         const uint32_t kw[4] = {kraw[u].x, kraw[u].y, kraw[u].z, kraw[u].w};
         const uint32_t sw[4] = {sraw[u].x, sraw[u].y, sraw[u].z, sraw[u].w};
 #pragma unroll
@@ -410,7 +416,7 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
         }
       }
     }
-    if (G > 1) part[tid] = pt;
+    if (G > 1 && done) part[tid] = pt;
   }
   __syncthreads();  // every state read above is complete before any state write below
 
@@ -521,6 +527,8 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
 __global__ void __launch_bounds__(kCompressThreads) compress_decode_kernel(CompressLaunch L) {
   __shared__ DecodePartial part[kCompressThreads];
   __shared__ float red[kCompressThreads / 32];
+  pdl_wait();
+  pdl_trigger();
   const CompressParams& P = blockIdx.y != 0 ? L.p[1] : L.p[0];
   const int b = blockIdx.x;
   if (b >= P.B) return;
@@ -535,6 +543,8 @@ __global__ void __launch_bounds__(kCompressThreads) compress_decode_kernel(Compr
 
 // Final state of a multi-token segment: one CTA per request, reads before writes.
 __global__ void __launch_bounds__(kCompressThreads) compress_state_kernel(CompressLaunch L) {
+  pdl_wait();
+  pdl_trigger();
   const CompressParams& P = L.p[blockIdx.z];
   const int b = blockIdx.x;
   if (b >= P.B) return;

@@ -45,21 +45,36 @@ __device__ __forceinline__ int visible_of(const IndexerParams& P, int b, int i) 
 }
 
 // Walks the work items [it, it1) that hold at least one visible entry, in order, and numbers
-// the query groups met (gi). Every role runs its own copy over the same range.
+// the query groups met (gi). Every role runs its own copy over the same range. The coordinates
+// advance incrementally (one division, at construction); the tiles of a group past its last
+// visible entry are skipped in one step.
 struct ItemIter {
   long long it, it1;
+  int et, qg, b;  // coordinates of item `it`
   int cur_b, cur_qg, gv, gi;
   bool started;
 
-  __device__ ItemIter(long long a, long long b) : it(a), it1(b), cur_b(-1), cur_qg(-1), gv(0), gi(-1), started(false) {}
+  __device__ ItemIter(const IndexerParams& P, long long a, long long e)
+      : it(a), it1(e), cur_b(-1), cur_qg(-1), gv(0), gi(-1), started(false) {
+    const long long gq = a / P.tiles_per_group;
+    et = (int)(a - gq * P.tiles_per_group);
+    b = (int)(gq / P.groups_per_req);
+    qg = (int)(gq - (long long)b * P.groups_per_req);
+  }
+
+  __device__ void next_group(const IndexerParams& P) {
+    et = 0;
+    if (++qg == P.groups_per_req) {
+      qg = 0;
+      ++b;
+    }
+  }
 
   __device__ bool next(const IndexerParams& P, ItemCoord& c, bool& new_group) {
     while (it < it1) {
-      const long long x = it++;
-      c.et = (int)(x % P.tiles_per_group);
-      const long long gq = x / P.tiles_per_group;
-      c.qg = (int)(gq % P.groups_per_req);
-      c.b = (int)(gq / P.groups_per_req);
+      c.et = et;
+      c.qg = qg;
+      c.b = b;
       if (c.b != cur_b || c.qg != cur_qg) {
         cur_b = c.b;
         cur_qg = c.qg;
@@ -68,7 +83,13 @@ struct ItemIter {
         const int i0 = c.qg * P.QG, i1 = min(P.S, i0 + P.QG);
         for (int i = i0; i < i1; ++i) gv = max(gv, visible_of(P, c.b, i));
       }
-      if (c.et * 128 >= gv) continue;
+      if (c.et * 128 >= gv) {  // nothing visible in the rest of this group
+        it += P.tiles_per_group - c.et;
+        next_group(P);
+        continue;
+      }
+      ++it;
+      if (++et == P.tiles_per_group) next_group(P);
       new_group = !started;
       if (new_group) {
         ++gi;
@@ -87,8 +108,6 @@ struct IdxSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  float w[2][256];   // per epilogue group: w of the group's current queries
-  int vis[2][256];   // per epilogue group: visible entries of those queries
 };
 
 template <int HI>
@@ -144,6 +163,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   uint8_t* k_tiles = base;                       // NS x 32 KB: [2 d-blocks][128 rows][128 B]
   uint8_t* q_tiles = base + (size_t)NS * 32768;  // 2 x q_bytes: [2 d-blocks][N rows][128 B]
   IdxSmem& sm = *reinterpret_cast<IdxSmem*>(q_tiles + 2 * (size_t)q_bytes);
+  // Per epilogue group: w of the group's current queries (N floats) and their visible entries.
+  float* w_arr = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(IdxSmem));
+  int* vis_arr = reinterpret_cast<int*>(w_arr + 2 * N);
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -178,6 +200,8 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x == 0) trace_time(P.status, 599);
 
   const long long total = P.total_items;
@@ -190,7 +214,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      ItemIter iter(it0, it1);
+      ItemIter iter(P, it0, it1);
       ItemCoord c;
       bool ng;
       long long n = 0;
@@ -221,7 +245,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, N, 0, 0);
-      ItemIter iter(it0, it1);
+      ItemIter iter(P, it0, it1);
       ItemCoord c;
       bool ng;
       long long n = 0;
@@ -266,9 +290,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     const int gt = threadIdx.x - 64 - 128 * grp;      // 0..127 within the group
     const int quad = warp & 3;                        // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
-    float* w_s = sm.w[grp];
-    int* vis_s = sm.vis[grp];
-    ItemIter iter(it0, it1);
+    float* w_s = w_arr + grp * N;
+    int* vis_s = vis_arr + grp * N;
+    ItemIter iter(P, it0, it1);
     ItemCoord c;
     bool ng;
     long long n = 0;
@@ -307,7 +331,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 }
 
 size_t indexer_smem_bytes(int stages, int N) {
-  return 1024 + (size_t)stages * 32768 + 2 * (size_t)N * 256 + sizeof(IdxSmem);
+  return 1024 + (size_t)stages * 32768 + 2 * (size_t)N * 256 + sizeof(IdxSmem) + 2 * 2 * (size_t)N * 4;
 }
 
 template __global__ void indexer_kernel<4>(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,

@@ -99,7 +99,7 @@ __global__ void topk_merge_kernel(TopkParams P);
 
 // ------------------------------------------------------------------------------ attention (K4/K5)
 
-constexpr int kAttnThreads = 416;         // warps 0..3 gathers, warp 4 MMA, warps 5..12 softmax
+constexpr int kAttnThreads = 288;         // warps 0..3 gathers, 4 MMA, 5..8 softmax
 constexpr int kAttnMaxWindow = 1024;
 constexpr int kAttnMaxTopk = 2048;
 constexpr int kAttnMaxCompressed = 2048;  // HCA: visible entries read per query

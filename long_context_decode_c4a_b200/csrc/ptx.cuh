@@ -25,6 +25,13 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Programmatic dependent launch. pdl_wait: wait until the grid this one depends on has completed
+// and its memory is visible (a no-op when the launch carries no such dependency); every thread
+// calls it before touching global memory another grid may still read or write. pdl_trigger:
+// allow the next grid on the stream to start launching (its threads still block in pdl_wait).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------------------
 // mbarrier
 
@@ -50,6 +57,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking test whether the phase of `bar` with the given parity has completed.
+__device__ __forceinline__ bool mbar_test(uint32_t bar_addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar_addr), "r"(parity)
@@ -151,10 +171,38 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_
                : "memory");
 }
 
+// Asynchronous 16-byte store into shared memory of a CTA of the cluster; the bytes are counted
+// (complete_tx) on that CTA's mbarrier `mbar_cluster`. Both addresses come from mapa_shared.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t mbar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   addr),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(mbar_cluster)
+               : "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster (address from mapa_shared), releasing this
 // thread's earlier writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Relaxed arrive on an mbarrier of another CTA of the cluster: it orders nothing, so it only
+// signals that this thread finished READING data the other CTA may now overwrite (the values
+// read were already consumed by earlier instructions, so those reads are complete).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory to shared memory of a CTA
+// of the cluster (dst and the mbarrier are cluster addresses from mapa_shared); the bytes are
+// counted (complete_tx) on that CTA's mbarrier. The source is read through the async proxy.
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst_cluster, uint32_t src_smem, uint32_t bytes,
+                                                     uint32_t mbar_cluster) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(src_smem), "r"(bytes), "r"(mbar_cluster)
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------------------------

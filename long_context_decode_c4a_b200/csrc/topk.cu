@@ -16,6 +16,7 @@
 // order, so the global top-k is contained in the union of the chunks' top-k lists.
 
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace csa {
 
@@ -50,9 +51,12 @@ struct Threshold {
 // splits the current range into at most kSelBins equal power-of-two bins, counts the keys of the
 // range per bin, and narrows the range to the bin that holds the krem-th largest key. A range of
 // up to 2^32 keys needs at most three passes (bin widths <= 2^21, <= 2^10, 1). `each(f)` calls
-// f(key) for every key the calling thread owns; all threads of the block must call this.
+// f(key) for every key the calling thread owns; all threads of the block call these together.
+
+// Count, minimum and maximum of the nonzero keys of the block.
 template <class ForEach>
-__device__ Threshold select_threshold(int k, ForEach each, SelectShared& sh) {
+__device__ __forceinline__ void select_stats(ForEach each, SelectShared& sh, uint32_t& total, uint32_t& lo,
+                                             uint32_t& hi) {
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
   uint32_t c = 0, mn = 0xFFFFFFFFu, mx = 0u;
   each([&](uint32_t key) {
@@ -74,12 +78,63 @@ __device__ Threshold select_threshold(int k, ForEach each, SelectShared& sh) {
     sh.wred[w][2] = mx;
   }
   __syncthreads();
-  uint32_t total = 0, lo = 0xFFFFFFFFu, hi = 0u;
+  total = 0;
+  lo = 0xFFFFFFFFu;
+  hi = 0u;
   for (int i = 0; i < nw; ++i) {
     total += sh.wred[i][0];
     lo = min(lo, sh.wred[i][1]);
     hi = max(hi, sh.wred[i][2]);
   }
+  __syncthreads();  // wred is reused by the first pass
+}
+
+// One pass: narrow [lo, hi] (lo < hi) to the bin holding the krem-th largest key of the range.
+template <class ForEach>
+__device__ __forceinline__ void select_pass(ForEach each, SelectShared& sh, uint32_t& lo, uint32_t& hi,
+                                            uint32_t& krem) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const uint32_t range = hi - lo;
+  const int shift = range < (uint32_t)kSelBins ? 0 : (32 - __clz((int)range)) - kSelBits;
+  const int nb = (int)(range >> shift) + 1;
+  const uint32_t l0 = lo, h0r = hi;
+  for (int i = tid; i < nb; i += blockDim.x) sh.hist[i] = 0u;
+  __syncthreads();
+  each([&](uint32_t key) {
+    if (key >= l0 && key <= h0r) atomicAdd(&sh.hist[(key - l0) >> shift], 1u);
+  });
+  __syncthreads();
+  // Thread t owns bins nb-1-2t and nb-2-2t: a scan in thread order runs over descending bins.
+  const int b0 = nb - 1 - 2 * tid, b1 = b0 - 1;
+  const uint32_t h0 = b0 >= 0 ? sh.hist[b0] : 0u, h1 = b1 >= 0 ? sh.hist[b1] : 0u;
+  const uint32_t s = h0 + h1;
+  uint32_t incl = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) sh.wred[w][0] = incl;
+  __syncthreads();
+  uint32_t excl = incl - s;
+  for (int i = 0; i < w; ++i) excl += sh.wred[i][0];
+  if (excl < krem && excl + s >= krem) {
+    const bool first = excl + h0 >= krem;
+    sh.bin = (uint32_t)(first ? b0 : b1);
+    sh.above = first ? excl : excl + h0;
+  }
+  __syncthreads();
+  krem -= sh.above;
+  const uint32_t nlo = lo + (sh.bin << shift);
+  hi = min(hi, nlo + ((1u << shift) - 1u));
+  lo = nlo;
+  __syncthreads();  // sh.bin / sh.above / wred are rewritten by the next pass
+}
+
+template <class ForEach>
+__device__ Threshold select_threshold(int k, ForEach each, SelectShared& sh) {
+  uint32_t total, lo, hi;
+  select_stats(each, sh, total, lo, hi);
   Threshold r;
   if (total <= (uint32_t)k) {
     r.take_all = true;
@@ -88,41 +143,7 @@ __device__ Threshold select_threshold(int k, ForEach each, SelectShared& sh) {
     return r;
   }
   uint32_t krem = (uint32_t)k;  // rank of T counted from the top of [lo, hi]
-  while (lo != hi) {
-    const uint32_t range = hi - lo;
-    const int shift = range < (uint32_t)kSelBins ? 0 : (32 - __clz((int)range)) - kSelBits;
-    const int nb = (int)(range >> shift) + 1;
-    for (int i = tid; i < nb; i += blockDim.x) sh.hist[i] = 0u;
-    __syncthreads();
-    each([&](uint32_t key) {
-      if (key >= lo && key <= hi) atomicAdd(&sh.hist[(key - lo) >> shift], 1u);
-    });
-    __syncthreads();
-    // Thread t owns bins nb-1-2t and nb-2-2t: a scan in thread order runs over descending bins.
-    const int b0 = nb - 1 - 2 * tid, b1 = b0 - 1;
-    const uint32_t h0 = b0 >= 0 ? sh.hist[b0] : 0u, h1 = b1 >= 0 ? sh.hist[b1] : 0u;
-    const uint32_t s = h0 + h1;
-    uint32_t incl = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (lane == 31) sh.wred[w][0] = incl;
-    __syncthreads();
-    uint32_t excl = incl - s;
-    for (int i = 0; i < w; ++i) excl += sh.wred[i][0];
-    if (excl < krem && excl + s >= krem) {
-      const bool first = excl + h0 >= krem;
-      sh.bin = (uint32_t)(first ? b0 : b1);
-      sh.above = first ? excl : excl + h0;
-    }
-    __syncthreads();
-    krem -= sh.above;
-    const uint32_t nlo = lo + (sh.bin << shift);
-    hi = min(hi, nlo + ((1u << shift) - 1u));
-    lo = nlo;
-  }
+  while (lo != hi) select_pass(each, sh, lo, hi, krem);
   r.take_all = false;
   r.T = lo;
   r.need = krem;
@@ -207,98 +228,106 @@ __device__ uint32_t block_topk(int n, int k, KeyFn key_of, EmitFn emit, TopkShar
   return tot_gt + min(tot_eq, th.need);
 }
 
-constexpr int kRegKeys = kTopkChunk / kTopkThreads;   // keys per thread in the chunk kernel (16)
+constexpr int kCandCap = 4096;   // keys of the threshold bin after the first pass, kept in smem
 
 struct TopkRegShared {
-  SelectShared sel;
-  uint32_t cnt[kRegKeys][32][2];   // per (key slot, warp): count of keys > T, == T
-  uint32_t off[kRegKeys][32][2];   // exclusive prefix over warps
-  uint32_t base[kRegKeys][2];      // keys > T / == T in all earlier key slots
-  uint32_t above, total;
+  TopkShared t;
+  uint32_t cand[kCandCap];
+  uint32_t ncand;
 };
 
-// Top-k of up to kRegKeys * blockDim keys held in registers (0 = empty position). Thread t holds
-// the keys of positions i = r * blockDim + t (r = 0 .. kRegKeys-1). Chosen positions are passed to
-// emit(pos, r) with pos = 0, 1, ... in increasing i. Returns the count.
-template <class EmitFn>
-__device__ uint32_t block_topk_regs(const uint32_t (&key)[kRegKeys], int k, EmitFn emit, TopkRegShared& sh) {
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
-  const Threshold th = select_threshold(k, [&](auto&& f) {
+// Top-k of up to KPT * blockDim keys held in registers (0 = empty position); thread t holds the
+// keys of positions t*KPT .. t*KPT+KPT-1. The first radix pass runs over the registers; the keys
+// left in the threshold bin (usually a few dozen) are then gathered into shared memory and the
+// remaining passes run over that list. Chosen positions are passed to emit(pos, r) (r = slot in
+// the thread's registers) with pos = 0, 1, ... in increasing position. Returns the count.
+template <int KPT, class EmitFn>
+__device__ uint32_t block_topk_regs(const uint32_t (&key)[KPT], int k, EmitFn emit, TopkRegShared& sh) {
+  const int tid = threadIdx.x, lane = tid & 31;
+  auto regs = [&](auto&& f) {
 #pragma unroll
-    for (int r = 0; r < kRegKeys; ++r) f(key[r]);
-  }, sh.sel);
-  // Compaction in index order: keep every key > T and the first `need` keys == T.
-  const uint32_t T = th.T;
-  const uint32_t need = th.need;
-  const bool take_all = th.take_all;
-  const uint32_t lt = (1u << lane) - 1u;
+    for (int r = 0; r < KPT; ++r) f(key[r]);
+  };
+  uint32_t total, lo, hi;
+  select_stats(regs, sh.t.sel, total, lo, hi);
+  const bool take_all = total <= (uint32_t)k;
+  uint32_t krem = (uint32_t)k;
+  if (!take_all && lo != hi) {
+    select_pass(regs, sh.t.sel, lo, hi, krem);
+    if (lo != hi) {
+      if (tid == 0) sh.ncand = 0;
+      __syncthreads();
+      const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int r = 0; r < kRegKeys; ++r) {
-    const bool gt = take_all ? key[r] != 0u : key[r] > T;
-    const bool eq = !take_all && key[r] == T;
-    const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
-    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) {
-      sh.cnt[r][w][0] = __popc(bgt);
-      sh.cnt[r][w][1] = __popc(beq);
+      for (int r = 0; r < KPT; ++r) {
+        const bool in = key[r] >= lo && key[r] <= hi;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        uint32_t base = 0;
+        if (lane == 0 && m != 0u) base = atomicAdd(&sh.ncand, (uint32_t)__popc(m));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        const uint32_t pos = base + (uint32_t)__popc(m & lt);
+        if (in && pos < (uint32_t)kCandCap) sh.cand[pos] = key[r];
+      }
+      __syncthreads();
+      const uint32_t nc = sh.ncand;
+      if (nc <= (uint32_t)kCandCap) {
+        auto list = [&](auto&& f) {
+          for (uint32_t i = tid; i < nc; i += blockDim.x) f(sh.cand[i]);
+        };
+        while (lo != hi) select_pass(list, sh.t.sel, lo, hi, krem);
+      } else {
+        while (lo != hi) select_pass(regs, sh.t.sel, lo, hi, krem);
+      }
     }
   }
-  __syncthreads();
-  if (w == 0) {
-    uint32_t run0 = 0, run1 = 0;
-    for (int r = 0; r < kRegKeys; ++r) {
-      uint32_t v0 = lane < nw ? sh.cnt[r][lane][0] : 0u, v1 = lane < nw ? sh.cnt[r][lane][1] : 0u;
-      uint32_t i0 = v0, i1 = v1;
+  // Compaction in position order: keep every key > T and the first `need` keys == T.
+  const uint32_t T = take_all ? 1u : lo;
+  const uint32_t need = take_all ? 0u : krem;
+  uint32_t n_gt = 0, n_eq = 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y0 = __shfl_up_sync(0xffffffffu, i0, o), y1 = __shfl_up_sync(0xffffffffu, i1, o);
-        if (lane >= o) {
-          i0 += y0;
-          i1 += y1;
-        }
-      }
-      if (lane < nw) {
-        sh.off[r][lane][0] = i0 - v0;
-        sh.off[r][lane][1] = i1 - v1;
-      }
-      if (lane == 0) {
-        sh.base[r][0] = run0;
-        sh.base[r][1] = run1;
-      }
-      run0 += __shfl_sync(0xffffffffu, i0, 31);
-      run1 += __shfl_sync(0xffffffffu, i1, 31);
-    }
-    if (lane == 0) {
-      sh.above = run0;   // keys > T
-      sh.total = run1;   // keys == T
+  for (int r = 0; r < KPT; ++r) {
+    if (key[r] == 0u) continue;
+    if (take_all || key[r] > T) ++n_gt;
+    else if (key[r] == T) ++n_eq;
+  }
+  uint32_t pre_gt, pre_eq, tot_gt, tot_eq;
+  block_scan2(n_gt, n_eq, sh.t, pre_gt, pre_eq, tot_gt, tot_eq);
+  uint32_t eq_seen = pre_eq;                       // keys == T before this thread's range
+  uint32_t pos = pre_gt + min(pre_eq, need);       // output slot of the next chosen key
+#pragma unroll
+  for (int r = 0; r < KPT; ++r) {
+    if (key[r] == 0u) continue;
+    if (take_all || key[r] > T) {
+      emit(pos++, r);
+    } else if (key[r] == T) {
+      if (eq_seen < need) emit(pos++, r);
+      ++eq_seen;
     }
   }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < kRegKeys; ++r) {
-    const bool gt = take_all ? key[r] != 0u : key[r] > T;
-    const bool eq = !take_all && key[r] == T;
-    const uint32_t bgt = __ballot_sync(0xffffffffu, gt);
-    const uint32_t beq = __ballot_sync(0xffffffffu, eq);
-    if (!(gt || eq)) continue;
-    const uint32_t gt_before = sh.base[r][0] + sh.off[r][w][0] + __popc(bgt & lt);
-    const uint32_t eq_before = sh.base[r][1] + sh.off[r][w][1] + __popc(beq & lt);
-    if (gt) {
-      emit(gt_before + min(eq_before, need), r);
-    } else if (eq_before < need) {
-      emit(gt_before + eq_before, r);
-    }
-  }
-  return sh.above + min(sh.total, need);
+  return tot_gt + min(tot_eq, need);
 }
 
-}  // namespace
+// Loads the keys of positions [t*KPT, t*KPT+KPT) of a score row of n entries (0 past the end).
+template <int KPT>
+__device__ __forceinline__ void load_keys(const float* row, int n, bool vec, uint32_t (&key)[KPT]) {
+  const int p0 = (int)threadIdx.x * KPT;
+  if (vec && p0 + KPT <= n) {
+#pragma unroll
+    for (int v = 0; v < KPT / 4; ++v) {
+      const float4 f = reinterpret_cast<const float4*>(row + p0)[v];
+      key[4 * v + 0] = score_key(f.x);
+      key[4 * v + 1] = score_key(f.y);
+      key[4 * v + 2] = score_key(f.z);
+      key[4 * v + 3] = score_key(f.w);
+    }
+  } else {
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) key[r] = p0 + r < n ? score_key(row[p0 + r]) : 0u;
+  }
+}
 
-// One CTA per (query, chunk). Chunk c of query q covers entries [c*chunk, min(E, (c+1)*chunk)).
-// Single-chunk queries write the final list; otherwise the chunk's top-k (key, index) pairs go to
-// the candidate buffers for topk_merge_kernel.
-__global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) {
-  __shared__ TopkRegShared sh;
+template <int KPT>
+__device__ void topk_chunk(const TopkParams& P, TopkRegShared& sh) {
   const int q = blockIdx.y;
   const int c = blockIdx.x;
   const int t = P.q_pos[q];
@@ -320,27 +349,36 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
     return;
   }
   const float* row = P.scores + (long long)q * P.scores_stride + lo;
-  uint32_t key[kRegKeys];
-#pragma unroll
-  for (int r = 0; r < kRegKeys; ++r) {
-    const int i = r * (int)blockDim.x + (int)threadIdx.x;
-    key[r] = i < n ? score_key(row[i]) : 0u;
-  }
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
+  uint32_t key[KPT];
+  load_keys<KPT>(row, n, vec, key);
+  const int p0 = lo + (int)threadIdx.x * KPT;
   if (nchunks <= 1) {
-    const uint32_t cnt = block_topk_regs(key, P.topk, [&](uint32_t pos, int r) {
-      out[pos] = lo + r * (int)blockDim.x + (int)threadIdx.x;
-    }, sh);
+    const uint32_t cnt = block_topk_regs<KPT>(key, P.topk, [&](uint32_t pos, int r) { out[pos] = p0 + r; }, sh);
     for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
   } else {
     const long long cb = ((long long)q * P.max_chunks + c) * P.topk;
     uint32_t* ck = P.cand_key + cb;
     int32_t* ci = P.cand_idx + cb;
-    const uint32_t cnt = block_topk_regs(key, P.topk, [&](uint32_t pos, int r) {
+    const uint32_t cnt = block_topk_regs<KPT>(key, P.topk, [&](uint32_t pos, int r) {
       ck[pos] = key[r];
-      ci[pos] = lo + r * (int)blockDim.x + (int)threadIdx.x;
+      ci[pos] = p0 + r;
     }, sh);
     if (threadIdx.x == 0) P.cand_cnt[(long long)q * P.max_chunks + c] = (int)cnt;
   }
+}
+
+}  // namespace
+
+// One CTA per (query, chunk). Chunk c of query q covers entries [c*chunk, min(E, (c+1)*chunk)).
+// Single-chunk queries write the final list; otherwise the chunk's top-k (key, index) pairs go to
+// the candidate buffers for topk_merge_kernel.
+__global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) {
+  __shared__ TopkRegShared sh;
+  pdl_wait();
+  pdl_trigger();
+  if (P.max_entries <= 8 * kTopkThreads) topk_chunk<8>(P, sh);  // rows of <= 8192 entries: 8 keys per thread
+  else topk_chunk<kTopkChunk / kTopkThreads>(P, sh);
 }
 
 // One CTA per query with more than one chunk: top-k over the union of the chunks' lists. The
@@ -349,6 +387,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
 __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) {
   __shared__ TopkShared sh;
   __shared__ int cnts[kTopkMaxChunks];
+  pdl_wait();
+  pdl_trigger();
   const int q = blockIdx.x;
   const int t = P.q_pos[q];
   int E = (t + 1) / P.ratio;

@@ -203,6 +203,14 @@ class CsaDecodeState:
         return decode_fused(self, pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink, out, cache_f32,
                             stage_events)
 
+    def prepare(self, pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink, out=None,
+                cache_f32=None) -> "PreparedDecode":
+        """Check and pack the arguments of step() once for repeated launches on fixed buffers."""
+        a, out = _csa_decode_args(self, pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink, out,
+                                  cache_f32)
+        keep = (self, pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink, cache_f32, out)
+        return PreparedDecode("csa_decode_fused", 5, a, keep)
+
 
 def _event_array(events, n: int):
     """ctypes array of the raw cudaEvent_t handles of n recorded torch.cuda.Event objects."""
@@ -216,9 +224,8 @@ def _event_array(events, n: int):
     return (ctypes.c_void_p * n)(*[e.cuda_event for e in events])
 
 
-def decode_fused(st: "CsaDecodeState", pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink,
-                 out: Optional[torch.Tensor] = None, cache_f32: Optional[torch.Tensor] = None,
-                 stage_events=None) -> torch.Tensor:
+def _csa_decode_args(st: "CsaDecodeState", pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink,
+                     out: Optional[torch.Tensor], cache_f32: Optional[torch.Tensor]):
     B, H, d, H_I, d_I = st.B, st.H, st.d, st.H_I, st.d_I
     _need(pos, "pos", torch.int32, (B,))
     _need(kv, "kv", torch.bfloat16, (B, 2 * d))
@@ -253,6 +260,33 @@ def decode_fused(st: "CsaDecodeState", pos, kv, score, idx_kv, idx_score, win_kv
     a.cache_f32 = _ptr(cache_f32)
     a.out, a.out_is_f32 = out.data_ptr(), int(out.dtype == torch.float32)
     a.ws, a.ws_bytes = st.ws.data_ptr(), st.ws.numel()
+    return a, out
+
+
+class PreparedDecode:
+    """One decode step whose arguments were checked and packed once: launch() enqueues it again
+    on the current stream with the same buffers (the caller refreshes their contents). It keeps
+    the tensors it points to alive."""
+
+    def __init__(self, fn_name: str, n_events: int, args, keep):
+        self._fn = getattr(_lib.load(), fn_name)
+        self._name = fn_name
+        self._n_events = n_events
+        self._a = args
+        self._keep = keep
+        self.out = keep[-1]
+
+    def launch(self, stage_events=None) -> torch.Tensor:
+        evs = _event_array(stage_events, self._n_events)
+        self._a.stage_events = ctypes.cast(evs, ctypes.c_void_p) if evs is not None else None
+        check(self._fn(ctypes.byref(self._a), _stream()), self._name)
+        return self.out
+
+
+def decode_fused(st: "CsaDecodeState", pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink,
+                 out: Optional[torch.Tensor] = None, cache_f32: Optional[torch.Tensor] = None,
+                 stage_events=None) -> torch.Tensor:
+    a, out = _csa_decode_args(st, pos, kv, score, idx_kv, idx_score, win_kv, q, q_idx, w, sink, out, cache_f32)
     evs = _event_array(stage_events, 5)
     a.stage_events = ctypes.cast(evs, ctypes.c_void_p) if evs is not None else None
     check(_lib.load().csa_decode_fused(ctypes.byref(a), _stream()), "csa_decode_fused")
@@ -279,9 +313,14 @@ class HcaDecodeState:
     def step(self, pos, kv, score, win_kv, q, sink, out=None, cache_f32=None, stage_events=None):
         return hca_decode_fused(self, pos, kv, score, win_kv, q, sink, out, cache_f32, stage_events)
 
+    def prepare(self, pos, kv, score, win_kv, q, sink, out=None, cache_f32=None) -> "PreparedDecode":
+        """Check and pack the arguments of step() once for repeated launches on fixed buffers."""
+        a, out = _hca_decode_args(self, pos, kv, score, win_kv, q, sink, out, cache_f32)
+        keep = (self, pos, kv, score, win_kv, q, sink, cache_f32, out)
+        return PreparedDecode("hca_decode_fused", 3, a, keep)
 
-def hca_decode_fused(st: "HcaDecodeState", pos, kv, score, win_kv, q, sink, out=None, cache_f32=None,
-                     stage_events=None) -> torch.Tensor:
+
+def _hca_decode_args(st: "HcaDecodeState", pos, kv, score, win_kv, q, sink, out, cache_f32):
     B, H, d = st.B, st.H, st.d
     _need(pos, "pos", torch.int32, (B,))
     _need(kv, "kv", torch.bfloat16, (B, d))
@@ -292,6 +331,8 @@ def hca_decode_fused(st: "HcaDecodeState", pos, kv, score, win_kv, q, sink, out=
     if out is None:
         out = torch.empty(B, H, d, dtype=torch.bfloat16, device=q.device)
     _need(out, "out", out.dtype, (B, H, d))
+    if cache_f32 is not None:
+        _need(cache_f32, "cache_f32", torch.float32, st.cache.shape)
     a = HcaDecodeArgs()
     a.B, a.H, a.d, a.rope_dim, a.ratio, a.window = B, H, d, st.rope_dim, st.ratio, st.window
     a.rope_base, a.eps, a.scale = st.rope_base, st.eps, 1.0 / math.sqrt(d)
@@ -303,6 +344,12 @@ def hca_decode_fused(st: "HcaDecodeState", pos, kv, score, win_kv, q, sink, out=
     a.cache_f32 = _ptr(cache_f32)
     a.out, a.out_is_f32 = out.data_ptr(), int(out.dtype == torch.float32)
     a.ws, a.ws_bytes = st.ws.data_ptr(), st.ws.numel()
+    return a, out
+
+
+def hca_decode_fused(st: "HcaDecodeState", pos, kv, score, win_kv, q, sink, out=None, cache_f32=None,
+                     stage_events=None) -> torch.Tensor:
+    a, out = _hca_decode_args(st, pos, kv, score, win_kv, q, sink, out, cache_f32)
     evs = _event_array(stage_events, 3)
     a.stage_events = ctypes.cast(evs, ctypes.c_void_p) if evs is not None else None
     check(_lib.load().hca_decode_fused(ctypes.byref(a), _stream()), "hca_decode_fused")

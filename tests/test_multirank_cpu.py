@@ -1,0 +1,76 @@
+"""The multi-process path of bench.py on CPU: two gloo ranks, as torchrun would start them.
+
+Requests are sharded over ranks (every rank owns its own B requests, no data-path collective);
+the only collectives are the barrier around the timed region and the max over ranks of the step
+time. The reference arm runs on rank 0 alone.
+"""
+
+import argparse
+import contextlib
+import io
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank: int, world: int, port: int, q) -> None:
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port))
+    try:
+        import bench
+        from synth import WORKLOADS, make_inputs
+
+        w, r, _ = bench.dist_setup(world)
+        bench.barrier(w)
+        # The max over ranks of a per-rank time.
+        m = bench.max_over_ranks(1.5 * (rank + 1), w)
+        # Each rank draws its own requests: the shard seeds differ by rank.
+        wl = WORKLOADS["pro_csa_decode_32k"].scaled(B=1)
+        x = make_inputs(wl, seed=wl.seed + 1000 * rank)
+        digest = float(x["q"].float().sum())
+        # The reference arm: rank 0 prints one JSON line, the others return without output.
+        args = argparse.Namespace(warmup=3, steps=1)
+        out = io.StringIO()
+        with contextlib.redirect_stdout(out):
+            rc = bench.run_reference(wl, args)
+        bench.barrier(w)
+        import torch.distributed as dist
+        dist.destroy_process_group()
+        q.put((rank, w, r, m, digest, rc, out.getvalue()))
+    except Exception as e:  # noqa: BLE001
+        q.put((rank, "error", repr(e)))
+
+
+@pytest.mark.timeout(600)
+def test_two_gloo_ranks_shard_requests_and_reduce_time():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        item = q.get(timeout=500)
+        res[item[0]] = item
+    for p in procs:
+        p.join(timeout=60)
+    for r in range(world):
+        assert res[r][1] != "error", res[r]
+        _, w, rr, m, digest, rc, out = res[r]
+        assert (w, rr, rc) == (world, r, 0)
+        assert m == pytest.approx(3.0)                     # max over ranks of 1.5 * (rank + 1)
+    assert res[0][4] != res[1][4], "the two ranks drew the same requests"
+    line = res[0][6].strip().splitlines()
+    assert len(line) == 1 and '"impl": "reference"' in line[0]
+    assert res[1][6].strip() == ""
