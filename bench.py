@@ -183,7 +183,7 @@ def step_inputs(inp):
             for k in keys if k in inp}
 
 
-def run_ours_decode(wl, args, world, rank):
+def run_ours_decode(wl, args, world, rank, light: bool = False):
     from long_context_decode_c4a_b200 import ops
     dev = torch.device("cuda")
     csa = wl.has_indexer
@@ -285,47 +285,164 @@ def run_ours_decode(wl, args, world, rank):
     stage_ms = {n: statistics.mean(stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(args.steps))
                 for i, n in enumerate(stage_names)}
 
-    # ---- end-to-end through the public API with host buffers
+    launches_per_step = (4 + (1 if wl.max_entries > 16384 else 0)) if csa else 2
+    if light:
+        return dict(ms=ms, stage_ms=stage_ms, clocks=clk, launches=launches_per_step * args.steps)
+    # ---- end-to-end through the public API with host buffers: every step copies its inputs from
+    # pinned host memory, runs, and copies its output back. Copies run on their own streams and
+    # overlap the neighbouring steps' compute (two device buffer sets, events between streams).
     st, x = sets[0]
     host = {k: v.to("cpu").pin_memory() for k, v in x.items() if k not in ("out", "sink")}
-    out_host = torch.empty(x["out"].shape, dtype=x["out"].dtype).pin_memory()
+    out_host = [torch.empty(x["out"].shape, dtype=x["out"].dtype).pin_memory() for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = out_host.numel() * out_host.element_size()
-    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
-
-    e2e_preps = []
-    for stt, xx in sets:
-        xin = dict(xx)
-        xin.update(dev_in)
-        if csa:
-            e2e_preps.append(stt.prepare(xin["pos"], xin["kv"], xin["score"], xin["idx_kv"], xin["idx_score"],
-                                         xin["win_kv"], xin["q"], xin["q_idx"], xin["w"], xin["sink"],
-                                         out=xin["out"]))
-        else:
-            e2e_preps.append(stt.prepare(xin["pos"], xin["kv"], xin["score"], xin["win_kv"], xin["q"], xin["sink"],
-                                         out=xin["out"]))
+    d2h = out_host[0].numel() * out_host[0].element_size()
+    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
+    dev_out = [torch.empty_like(x["out"]) for _ in range(2)]
+    e2e_preps = []   # [buffer][input set]
+    for buf in range(2):
+        row = []
+        for stt, xx in sets:
+            xin = dict(xx)
+            xin.update(dev_in[buf])
+            if csa:
+                row.append(stt.prepare(xin["pos"], xin["kv"], xin["score"], xin["idx_kv"], xin["idx_score"],
+                                       xin["win_kv"], xin["q"], xin["q_idx"], xin["w"], xin["sink"],
+                                       out=dev_out[buf]))
+            else:
+                row.append(stt.prepare(xin["pos"], xin["kv"], xin["score"], xin["win_kv"], xin["q"], xin["sink"],
+                                       out=dev_out[buf]))
+        e2e_preps.append(row)
+    comp = torch.cuda.current_stream()
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+    for e in comp_done + d2h_done:
+        e.record(comp)
 
     def e2e_step(i):
-        for k, v in host.items():
-            dev_in[k].copy_(v, non_blocking=True)
-        out = e2e_preps[i % len(e2e_preps)].launch()
-        out_host.copy_(out, non_blocking=True)
+        buf = i % 2
+        s_h2d.wait_event(comp_done[buf])          # step i-2 finished reading dev_in[buf]
+        with torch.cuda.stream(s_h2d):
+            for k, v in host.items():
+                dev_in[buf][k].copy_(v, non_blocking=True)
+            h2d_done[buf].record(s_h2d)
+        comp.wait_event(h2d_done[buf])
+        comp.wait_event(d2h_done[buf])             # step i-2's output was copied out of dev_out[buf]
+        e2e_preps[buf][i % len(sets)].launch()
+        comp_done[buf].record(comp)
+        s_d2h.wait_event(comp_done[buf])
+        with torch.cuda.stream(s_d2h):
+            out_host[buf].copy_(dev_out[buf], non_blocking=True)
+            d2h_done[buf].record(s_d2h)
 
     for i in range(args.warmup):
         e2e_step(i)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(s_h2d)
     for k in range(args.steps):
         e2e_step(k)
-    e1.record()
+    s_h2d.wait_stream(s_d2h)
+    e1.record(s_h2d)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    launches_per_step = (4 + (1 if wl.max_entries > 16384 else 0)) if csa else 2
     return dict(ms=ms, stage_ms=stage_ms, clocks=clk, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
                 launches=launches_per_step * args.steps)
+
+
+def prefill_ledger(wl):
+    """Algorithmic tensor FLOPs of one CSA prefill pass: attention 4*H*reads*d per query (the
+    pages' analytic count) plus the indexer's 2*H_I*d_I per (query, visible entry)."""
+    attn = idx = 0
+    for t in range(wl.S):
+        vis = min((t + 1) // wl.ratio, wl.max_entries)   # entries visible to query t
+        reads = min(wl.W, t + 1) + min(wl.topk, vis)      # window rows + selected entries
+        attn += 4 * wl.H * reads * wl.d
+        idx += 2 * wl.H_I * wl.d_I * vis
+    return attn, idx
+
+
+def run_prefill(wl, steps: int, warmup: int):
+    """One CSA prefill pass over S tokens from an empty cache, through the C ABI: both compressor
+    streams, indexer + top-k, sparse attention. Returns ms per pass and per stage."""
+    from long_context_decode_c4a_b200 import ops
+    dev = "cuda"
+    inp = make_inputs(wl, device=dev)
+    B, S, d, dI, E = wl.B, wl.S, wl.d, wl.d_I, wl.max_entries
+    main_cfg, idx_cfg = ops.compressor_cfg(4, d), ops.compressor_cfg(4, dI)
+    skv = torch.empty(B, 8, 2 * d, dtype=torch.bfloat16, device=dev)
+    ssc = torch.empty_like(skv)
+    ikv = torch.empty(B, 8, 2 * dI, dtype=torch.bfloat16, device=dev)
+    isc = torch.empty_like(ikv)
+    cache = torch.zeros(B, E, d, dtype=torch.bfloat16, device=dev)
+    icache = torch.zeros(B, E, dI, dtype=torch.bfloat16, device=dev)
+    start = torch.zeros(B, dtype=torch.int32, device=dev)
+    topk = torch.empty(B, S, wl.topk, dtype=torch.int32, device=dev)
+    out = torch.empty(B, S, wl.H, d, dtype=torch.bfloat16, device=dev)
+    ws_i = ops.workspace(ops._lib.CSA_WS_INDEXER_TOPK, B, S, E, wl.topk, dev)
+    ws_a = ops.workspace(ops._lib.CSA_WS_SPARSE_ATTN, B, S, E, wl.topk, dev)
+
+    def one(evs=None):
+        if evs:
+            evs[0].record()
+        ops.state_reset(main_cfg, skv, ssc)
+        ops.state_reset(idx_cfg, ikv, isc)
+        ops.compress(main_cfg, start, inp["kv"], inp["score"], inp["gamma"], skv, ssc, cache)
+        ops.compress(idx_cfg, start, inp["idx_kv"], inp["idx_score"], inp["idx_gamma"], ikv, isc, icache)
+        if evs:
+            evs[1].record()
+        ops.indexer_topk(inp["pos"], inp["q_idx"], inp["w"], icache, wl.topk, topk_idx=topk, ws=ws_i)
+        if evs:
+            evs[2].record()
+        ops.sparse_attn(inp["pos"], inp["q"], inp["win_kv"], cache, topk, inp["sink"], wl.W, out=out, ws=ws_a)
+        if evs:
+            evs[3].record()
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for k in range(steps):
+        one(evs[k])
+    torch.cuda.synchronize()
+    for w in (ws_i, ws_a):
+        if ops.device_status(w) != 0:
+            raise RuntimeError("device status after the prefill passes")
+    per = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
+    return dict(ms=per(0, 3), stage_ms={"compress": per(0, 1), "indexer_topk": per(1, 2), "attention": per(2, 3)})
+
+
+def extra_workloads(args, peaks):
+    """Short measurements of the other synthetic configurations (one GPU, same process)."""
+    res = {}
+    for name in ("pro_hca_decode_32k", "long_csa_decode_1m"):
+        wl = WORKLOADS[name]
+        a = argparse.Namespace(**vars(args))
+        a.steps, a.warmup, a.sets = 20, 3, 2 if name == "long_csa_decode_1m" else args.sets
+        r = run_ours_decode(wl, a, 1, 0, light=True)
+        per_q, reads = decode_bytes(wl)
+        total = sum(per_q.values()) * wl.B
+        res[name] = {"value": wl.B * 1000.0 / r["ms"], "unit": "queries/s", "tokens_per_s": wl.B * 1000.0 / r["ms"],
+                     "ms_per_step": r["ms"], "kernels_ms": r["stage_ms"], "reads_per_query": reads,
+                     "roofline": {"bound": "hbm", "achieved": total / (r["ms"] * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": total / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                  "scope": "whole step, algorithmic bytes"}}
+        torch.cuda.empty_cache()
+    for name, steps in (("csa_prefill_8k", 3), ("tiny_csa_prefill", 20)):
+        wl = WORKLOADS[name]
+        r = run_prefill(wl, steps, 3)
+        attn_f, idx_f = prefill_ledger(wl)
+        tf = (attn_f + idx_f) / (r["ms"] * 1e-3) / 1e12
+        res[name] = {"value": wl.B * wl.S * 1000.0 / r["ms"], "unit": "tokens/s", "ms_per_step": r["ms"],
+                     "kernels_ms": r["stage_ms"],
+                     "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                  "frac": tf / peaks["bf16_tflops"], "flops_per_pass": attn_f + idx_f,
+                                  "scope": "whole pass, algorithmic FLOPs (attention 4*H*reads*d + indexer)"}}
+        torch.cuda.empty_cache()
+    return res
 
 
 def oracle_decode_time(wl, n_req: int, seed: int = 1):
@@ -371,6 +488,7 @@ def main(argv=None):
     ap.add_argument("--sets", type=int, default=4, help="rotating input sets")
     ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the short runs of the other configurations")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch every timed step from the host instead of replaying a CUDA graph")
     args = ap.parse_args(argv)
@@ -431,6 +549,8 @@ def main(argv=None):
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
+    if world == 1 and not args.no_extra:
+        line["workloads"] = extra_workloads(args, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline_decode(wl)
     if rank == 0:

@@ -340,7 +340,8 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
   T.cand_cnt = reinterpret_cast<int*>(ws + L.cand_cnt_off);
   T.status = status;
   const int nchunks = std::max(1, L.max_chunks);
-  CSA_CUDA(launch_pdl(topk_chunk_kernel, dim3((unsigned)nchunks, (unsigned)queries), dim3(kTopkThreads), 0, st, T));
+  const int tk_threads = a.max_entries <= kTopkShortRow ? kTopkShortThreads : kTopkThreads;
+  CSA_CUDA(launch_pdl(topk_chunk_kernel, dim3((unsigned)nchunks, (unsigned)queries), dim3(tk_threads), 0, st, T));
   if (L.max_chunks > 1) {
     CSA_CHECK_SUP(L.max_chunks <= kTopkMaxChunks, "max_entries too large for the top-k merge");
     CSA_CUDA(launch_pdl(topk_merge_kernel, dim3((unsigned)queries), dim3(kTopkThreads), 0, st, T));

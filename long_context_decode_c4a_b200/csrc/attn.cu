@@ -22,8 +22,10 @@
 //     and PV as an MN-major B operand; Q[:, 0:256] passes through stages 2-3 on its way into
 //     TMEM); the candidate list.
 //   Warps: 0..3 build the candidate list and gather rows with coalesced 16-byte cp.async (then
-//     share the epilogue); 4 issues the MMAs (and owns TMEM); 5..8 run the softmax (thread = head
-//     = TMEM lane) and the epilogue.
+//     share the epilogue); 4 and 5 issue the score MMAs of even and odd tiles (one thread issues a
+//     tcgen05.mma only every ~50 cycles, so two issuers keep the tensor pipe fed); 6 issues the PV
+//     MMAs in tile order (and owns TMEM); 7..10 run the softmax (thread = head = TMEM lane) and the
+//     epilogue.
 // Precision: P = P_hi + P_lo with both parts in bf16 (about 16 significant bits), accumulated by two
 // PV MMAs; a single bf16 P (8 bits) leaves errors near 1% of the output RMS on short candidate sets.
 // Online softmax in the log2 domain; the running max starts at the sink; O is rescaled only when a
@@ -43,8 +45,9 @@ constexpr uint32_t kInvalid = 0x80000000u;    // list entry flag: padding slot (
 constexpr uint32_t kFromCache = 0x40000000u;  // list entry flag: row of the compressed cache
 constexpr uint32_t kRowMask = 0x3FFFFFFFu;
 constexpr int kProducers = 128;               // warps 0..3
-constexpr int kMmaWarp = 4;
-constexpr int kSoftWarp0 = 5;                 // warps 5..8
+constexpr int kQkWarp0 = 4;                   // warps 4, 5: score MMAs of even / odd tiles
+constexpr int kPvWarp = 6;                    // PV MMAs; owns TMEM
+constexpr int kSoftWarp0 = 7;                 // warps 7..10
 constexpr int kSoftThreads = 128;
 constexpr int kTile = 32;                     // candidates per tile
 constexpr int kStages = 4;
@@ -56,12 +59,15 @@ constexpr uint32_t kBlockBytes = 4096;        // one 64-dim block of a stage: [3
 static_assert(kAttnThreads == 32 * (kSoftWarp0 + 4), "warp roles");
 static_assert(kAttnMaxCands % kTile == 0, "candidate capacity");
 
+static_assert(kStages == kSBufs, "tile j uses stage and score tile j % kStages");
+
 struct AttnSmem {
   uint64_t q_full, q_done, list_ready;
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t kv_full[kStages];
+  uint64_t buf_free[kStages];         // PV(j) completed: stage and score tile j % kStages are free
   uint64_t s_full[kSBufs], p_full[kSBufs], o_done[2];
   uint64_t epi;                       // the softmax warps published 1/l
-  uint64_t drain;
+  uint64_t drain[3];
   uint32_t tmem_base;
   int abort_flag;
   int n_tiles;
@@ -77,6 +83,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
   return r;
+}
+
+// 2^x by the MUFU.EX2 unit (ex2.approx: about 2 ulp, 2^-inf = 0); its error is far below the
+// ~2^-16 relative precision that the P_hi + P_lo pair keeps.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -175,7 +189,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&sm.list_ready, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.kv_full[i], kProducers);
-      mbar_init(&sm.kv_empty[i], 1);
+      mbar_init(&sm.buf_free[i], 1);
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&sm.s_full[i], 1);
@@ -184,12 +198,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&sm.o_done[0], 1);
     mbar_init(&sm.o_done[1], 1);
     mbar_init(&sm.epi, kSoftThreads);
-    mbar_init(&sm.drain, 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&sm.drain[i], 1);
     sm.abort_flag = 0;
     sm.bad = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kPvWarp) {
     tmem_alloc(&sm.tmem_base, 512);
     tmem_relinquish();
   }
@@ -297,7 +311,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           break;
         }
       } else if (issue && next >= kStages) {
-        uint64_t* empty = &sm.kv_empty[next % kStages];
+        uint64_t* empty = &sm.buf_free[next % kStages];
         const uint32_t par = (uint32_t)((next / kStages - 1) & 1);
         if (next > ann) {
           issue = mbar_test(smem_u32(empty), par);
@@ -341,53 +355,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       store_rows(P, sm, tmem + ((uint32_t)(quad * 32) << 16) + 256, 128, half, (long long)qi * P.H + h, h,
                  sm.inv_l[h]);
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp < kPvWarp) {
+    // ------------------------------------------------------------ score MMAs: tiles j = w, w+2, ...
     if (lane == 0) {
+      const int w = warp - kQkWarp0;  // 0: even tiles, 1: odd tiles
       bool ok = mbar_wait(&sm.q_full, 0, abort_flag, status, 111) &&
                 mbar_wait(&sm.q_done, 0, abort_flag, status, 112) &&
                 mbar_wait(&sm.list_ready, 0, abort_flag, status, 113);
       const int J = ok ? sm.n_tiles : 0;
       const uint32_t idesc_qk = idesc_bf16_f32(128, kTile, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
       const uint32_t qhi = smem_u32(q_hi);
-      int pv_next = 0;
-      auto issue_pv = [&](int jj) -> bool {
-        const int sb = jj % kSBufs;
-        if (!mbar_wait(&sm.p_full[sb], (uint32_t)((jj / kSBufs) & 1), abort_flag, status, 115)) return false;
-        tc_fence_after();
-        const uint32_t vbase =
-            smem_u32(stage0 + (size_t)(jj % kStages) * kStageBytes) + (uint32_t)(4 * half) * kBlockBytes;
-        const uint32_t pcol = tmem + 128 + kTile * sb;
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {  // P_hi, then P_lo
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t bdesc = smem_desc_sw128(vbase + ks * 2048, kBlockBytes, 1024);
-            mma_ts(tmem + 256, pcol + 16 * part + 8 * ks, bdesc, idesc_pv, (jj > 0 || part > 0 || ks > 0) ? 1u : 0u);
-          }
-        }
-        mma_commit(&sm.o_done[jj & 1]);
-        mma_commit(&sm.kv_empty[jj % kStages]);
-        if (jj < 60) trace_time(status, 192 + jj);
-        return true;
-      };
-      int j = 0;
-      for (; j < J; ++j) {
-        // Score tile j % kSBufs is free once PV(j - kSBufs) has been issued (the tensor pipe runs
-        // in issue order); issue the PVs whose P is ready anyway.
-        bool okp = true;
-        while (okp && pv_next <= j - kSBufs) okp = issue_pv(pv_next++);
-        while (okp && pv_next < j &&
-               mbar_test(smem_u32(&sm.p_full[pv_next % kSBufs]), (uint32_t)((pv_next / kSBufs) & 1)))
-          okp = issue_pv(pv_next++);
-        if (!okp) break;
+      for (int j = w; j < J; j += 2) {
         const int s = j % kStages;
+        // Score tile s is rewritten only once PV(j - kStages), which read its P, has completed.
+        if (j >= kStages && !mbar_wait(&sm.buf_free[s], (uint32_t)((j / kStages - 1) & 1), abort_flag, status, 117))
+          break;
         if (!mbar_wait(&sm.kv_full[s], (uint32_t)((j / kStages) & 1), abort_flag, status, 114)) break;
         tc_fence_after();
         if (j < 60) trace_time(status, 64 + j);
         const uint32_t kbase = smem_u32(stage0 + (size_t)s * kStageBytes);
-        const uint32_t d_s = tmem + 128 + kTile * (j % kSBufs);
+        const uint32_t d_s = tmem + 128 + kTile * s;
 #pragma unroll
         for (int ks = 0; ks < 16; ++ks) {  // dims 0..255: A = Q from TMEM
           const uint64_t bdesc = smem_desc_sw128(kbase + (ks >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024);
@@ -399,15 +386,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const uint64_t bdesc = smem_desc_sw128(kbase + (ks >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024);
           mma_ss(d_s, adesc, bdesc, idesc_qk, 1u);
         }
-        mma_commit(&sm.s_full[j % kSBufs]);
-      }
-      if (j == J) {
-        bool okp = true;
-        while (okp && pv_next < J) okp = issue_pv(pv_next++);
+        mma_commit(&sm.s_full[s]);
       }
       // Every MMA issued above completes on its own; wait for them before TMEM is released.
-      mma_commit(&sm.drain);
-      mbar_wait_drain(&sm.drain, 0, status, 116);
+      mma_commit(&sm.drain[w]);
+      mbar_wait_drain(&sm.drain[w], 0, status, 116);
+    }
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ PV MMAs, in tile order
+    if (lane == 0) {
+      bool ok = mbar_wait(&sm.list_ready, 0, abort_flag, status, 118);
+      const int J = ok ? sm.n_tiles : 0;
+      const uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
+      for (int j = 0; j < J; ++j) {
+        const int sb = j % kSBufs;
+        if (!mbar_wait(&sm.p_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 115)) break;
+        tc_fence_after();
+        const uint32_t vbase =
+            smem_u32(stage0 + (size_t)(j % kStages) * kStageBytes) + (uint32_t)(4 * half) * kBlockBytes;
+        const uint32_t pcol = tmem + 128 + kTile * sb;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {  // P_hi, then P_lo
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t bdesc = smem_desc_sw128(vbase + ks * 2048, kBlockBytes, 1024);
+            mma_ts(tmem + 256, pcol + 16 * part + 8 * ks, bdesc, idesc_pv, (j > 0 || part > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&sm.o_done[j & 1]);
+        mma_commit(&sm.buf_free[j % kStages]);
+        if (j < 60) trace_time(status, 192 + j);
+      }
+      mma_commit(&sm.drain[2]);
+      mbar_wait_drain(&sm.drain[2], 0, status, 119);
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 5..8), epilogue
@@ -463,10 +474,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint32_t mk = sm.mask[j];
       float x[32];
       float mt = -CUDART_INF_F;
+      if (mk == 0xFFFFFFFFu) {  // a full tile (the common case): no padding to mask
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = ((mk >> c) & 1u) ? __uint_as_float(v[c]) * P.scale_log2 : -CUDART_INF_F;
-        mt = fmaxf(mt, x[c]);
+        for (int c = 0; c < 32; ++c) {
+          x[c] = __uint_as_float(v[c]) * P.scale_log2;
+          mt = fmaxf(mt, x[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[c] = ((mk >> c) & 1u) ? __uint_as_float(v[c]) * P.scale_log2 : -CUDART_INF_F;
+          mt = fmaxf(mt, x[c]);
+        }
       }
       // Lazy rescale: only when this tile raises the row max by more than 2^8. The TMEM accesses
       // are warp-collective, so the whole warp takes the branch if any lane needs it (lanes that do
@@ -501,8 +520,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float rs = 0.f;
 #pragma unroll
       for (int q = 0; q < 16; ++q) {
-        const float p0 = exp2f(x[2 * q] - m_used);
-        const float p1 = exp2f(x[2 * q + 1] - m_used);
+        const float p0 = ex2_approx(x[2 * q] - m_used);
+        const float p1 = ex2_approx(x[2 * q + 1] - m_used);
         phi[q] = pack_bf16(p0, p1);
         plo[q] = pack_bf16(p0 - bf16_lo(phi[q]), p1 - bf16_hi(phi[q]));
         rs += p0 + p1;
@@ -532,7 +551,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (threadIdx.x == 0) trace_time(status, 255);
-  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
+  if (warp == kPvWarp) tmem_dealloc(tmem, 512);
 }
 
 size_t attn_smem_bytes() { return 1024 + kQhiBytes + kStages * kStageBytes + sizeof(AttnSmem); }

@@ -78,6 +78,8 @@ __global__ void indexer_kernel(const __grid_constant__ CUtensorMap map_k, const 
 // ------------------------------------------------------------------------------ top-k (K3)
 
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkShortThreads = 1024;   // rows of <= kTopkShortRow entries: 1024 threads x 8 keys
+constexpr int kTopkShortRow = 8192;
 constexpr int kTopkChunk = 16384;         // entries per chunk (staged in 64 KB of smem)
 constexpr int kTopkMaxChunks = 1024;
 
@@ -99,7 +101,7 @@ __global__ void topk_merge_kernel(TopkParams P);
 
 // ------------------------------------------------------------------------------ attention (K4/K5)
 
-constexpr int kAttnThreads = 288;         // warps 0..3 gathers, 4 MMA, 5..8 softmax
+constexpr int kAttnThreads = 352;         // warps 0..3 gathers, 4-5 score MMAs, 6 PV MMAs, 7..10 softmax
 constexpr int kAttnMaxWindow = 1024;
 constexpr int kAttnMaxTopk = 2048;
 constexpr int kAttnMaxCompressed = 2048;  // HCA: visible entries read per query

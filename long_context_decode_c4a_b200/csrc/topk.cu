@@ -78,37 +78,24 @@ __device__ __forceinline__ void select_stats(ForEach each, SelectShared& sh, uin
     sh.wred[w][2] = mx;
   }
   __syncthreads();
-  total = 0;
-  lo = 0xFFFFFFFFu;
-  hi = 0u;
-  for (int i = 0; i < nw; ++i) {
-    total += sh.wred[i][0];
-    lo = min(lo, sh.wred[i][1]);
-    hi = max(hi, sh.wred[i][2]);
+  // Every warp reduces the per-warp partials with shuffles (lane i reads warp i's).
+  total = lane < nw ? sh.wred[lane][0] : 0u;
+  lo = lane < nw ? sh.wred[lane][1] : 0xFFFFFFFFu;
+  hi = lane < nw ? sh.wred[lane][2] : 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
   __syncthreads();  // wred is reused by the first pass
 }
 
-// One pass: narrow [lo, hi] (lo < hi) to the bin holding the krem-th largest key of the range.
-template <class ForEach>
-__device__ __forceinline__ void select_pass(ForEach each, SelectShared& sh, uint32_t& lo, uint32_t& hi,
-                                            uint32_t& krem) {
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const uint32_t range = hi - lo;
-  const int shift = range < (uint32_t)kSelBins ? 0 : (32 - __clz((int)range)) - kSelBits;
-  const int nb = (int)(range >> shift) + 1;
-  const uint32_t l0 = lo, h0r = hi;
-  for (int i = tid; i < nb; i += blockDim.x) sh.hist[i] = 0u;
-  __syncthreads();
-  each([&](uint32_t key) {
-    if (key >= l0 && key <= h0r) atomicAdd(&sh.hist[(key - l0) >> shift], 1u);
-  });
-  __syncthreads();
-  // Thread t owns bins nb-1-2t and nb-2-2t: a scan in thread order runs over descending bins.
-  const int b0 = nb - 1 - 2 * tid, b1 = b0 - 1;
-  const uint32_t h0 = b0 >= 0 ? sh.hist[b0] : 0u, h1 = b1 >= 0 ? sh.hist[b1] : 0u;
-  const uint32_t s = h0 + h1;
-  uint32_t incl = s;
+// Exclusive prefix (in thread order) and total of one count per thread; wred[*][0] is scratch.
+// All threads of the block call it; it ends with a barrier so wred can be reused.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, SelectShared& sh, uint32_t& total) {
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  uint32_t incl = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -116,19 +103,65 @@ __device__ __forceinline__ void select_pass(ForEach each, SelectShared& sh, uint
   }
   if (lane == 31) sh.wred[w][0] = incl;
   __syncthreads();
-  uint32_t excl = incl - s;
-  for (int i = 0; i < w; ++i) excl += sh.wred[i][0];
-  if (excl < krem && excl + s >= krem) {
-    const bool first = excl + h0 >= krem;
-    sh.bin = (uint32_t)(first ? b0 : b1);
-    sh.above = first ? excl : excl + h0;
+  uint32_t wv = lane < nw ? sh.wred[lane][0] : 0u;  // inclusive scan of the warp totals
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, wv, o);
+    if (lane >= o) wv += y;
+  }
+  total = __shfl_sync(0xffffffffu, wv, 31);
+  const uint32_t before = w == 0 ? 0u : __shfl_sync(0xffffffffu, wv, w - 1);
+  __syncthreads();
+  return before + incl - v;
+}
+
+// One pass: narrow [lo, hi] (lo < hi) to the bin holding the krem-th largest key of the range.
+// NT = threads of the block (each owns kSelBins / NT consecutive bins, in descending order).
+template <int NT, class ForEach>
+__device__ __forceinline__ void select_pass(ForEach each, SelectShared& sh, uint32_t& lo, uint32_t& hi,
+                                            uint32_t& krem) {
+  constexpr int BPT = kSelBins / NT;
+  static_assert(BPT * NT == kSelBins, "bins per thread");
+  const int tid = threadIdx.x;
+  const uint32_t range = hi - lo;
+  const int shift = range < (uint32_t)kSelBins ? 0 : (32 - __clz((int)range)) - kSelBits;
+  const int nb = (int)(range >> shift) + 1;
+  const uint32_t l0 = lo, h0r = hi;
+  for (int i = tid; i < nb; i += NT) sh.hist[i] = 0u;
+  __syncthreads();
+  each([&](uint32_t key) {
+    if (key >= l0 && key <= h0r) atomicAdd(&sh.hist[(key - l0) >> shift], 1u);
+  });
+  __syncthreads();
+  // Thread t owns bins nb-1-t*BPT down to nb-(t+1)*BPT: a scan in thread order runs over
+  // descending bins.
+  uint32_t hb[BPT];
+  uint32_t cnt = 0;
+#pragma unroll
+  for (int k = 0; k < BPT; ++k) {
+    const int bin = nb - 1 - tid * BPT - k;
+    hb[k] = bin >= 0 ? sh.hist[bin] : 0u;
+    cnt += hb[k];
+  }
+  uint32_t tot;
+  uint32_t run = block_excl_scan(cnt, sh, tot);
+  if (run < krem && run + cnt >= krem) {
+#pragma unroll
+    for (int k = 0; k < BPT; ++k) {
+      if (run + hb[k] >= krem) {
+        sh.bin = (uint32_t)(nb - 1 - tid * BPT - k);
+        sh.above = run;
+        break;
+      }
+      run += hb[k];
+    }
   }
   __syncthreads();
   krem -= sh.above;
   const uint32_t nlo = lo + (sh.bin << shift);
   hi = min(hi, nlo + ((1u << shift) - 1u));
   lo = nlo;
-  __syncthreads();  // sh.bin / sh.above / wred are rewritten by the next pass
+  __syncthreads();  // sh.bin / sh.above are rewritten by the next pass
 }
 
 template <class ForEach>
@@ -143,7 +176,7 @@ __device__ Threshold select_threshold(int k, ForEach each, SelectShared& sh) {
     return r;
   }
   uint32_t krem = (uint32_t)k;  // rank of T counted from the top of [lo, hi]
-  while (lo != hi) select_pass(each, sh, lo, hi, krem);
+  while (lo != hi) select_pass<1024>(each, sh, lo, hi, krem);
   r.take_all = false;
   r.T = lo;
   r.need = krem;
@@ -158,37 +191,8 @@ struct TopkShared {
 // Exclusive prefix of two per-thread counts across the block (thread order), and the totals.
 __device__ __forceinline__ void block_scan2(uint32_t a, uint32_t b, TopkShared& sh, uint32_t& pre_a, uint32_t& pre_b,
                                             uint32_t& tot_a, uint32_t& tot_b) {
-  const uint32_t lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  uint32_t ia = a, ib = b;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t ya = __shfl_up_sync(0xffffffffu, ia, o);
-    const uint32_t yb = __shfl_up_sync(0xffffffffu, ib, o);
-    if (lane >= (uint32_t)o) {
-      ia += ya;
-      ib += yb;
-    }
-  }
-  __syncthreads();
-  if (lane == 31) {
-    sh.warp_tot[w][0] = ia;
-    sh.warp_tot[w][1] = ib;
-  }
-  __syncthreads();
-  uint32_t oa = 0, ob = 0, ta = 0, tb = 0;
-  for (uint32_t i = 0; i < nw; ++i) {
-    const uint32_t xa = sh.warp_tot[i][0], xb = sh.warp_tot[i][1];
-    if (i < w) {
-      oa += xa;
-      ob += xb;
-    }
-    ta += xa;
-    tb += xb;
-  }
-  pre_a = oa + ia - a;
-  pre_b = ob + ib - b;
-  tot_a = ta;
-  tot_b = tb;
+  pre_a = block_excl_scan(a, sh.sel, tot_a);
+  pre_b = block_excl_scan(b, sh.sel, tot_b);
 }
 
 // Select the top k of the n keys key_of(i) (0 = empty position) with ties to the lower position,
@@ -241,7 +245,7 @@ struct TopkRegShared {
 // left in the threshold bin (usually a few dozen) are then gathered into shared memory and the
 // remaining passes run over that list. Chosen positions are passed to emit(pos, r) (r = slot in
 // the thread's registers) with pos = 0, 1, ... in increasing position. Returns the count.
-template <int KPT, class EmitFn>
+template <int NT, int KPT, class EmitFn>
 __device__ uint32_t block_topk_regs(const uint32_t (&key)[KPT], int k, EmitFn emit, TopkRegShared& sh) {
   const int tid = threadIdx.x, lane = tid & 31;
   auto regs = [&](auto&& f) {
@@ -253,7 +257,7 @@ __device__ uint32_t block_topk_regs(const uint32_t (&key)[KPT], int k, EmitFn em
   const bool take_all = total <= (uint32_t)k;
   uint32_t krem = (uint32_t)k;
   if (!take_all && lo != hi) {
-    select_pass(regs, sh.t.sel, lo, hi, krem);
+    select_pass<NT>(regs, sh.t.sel, lo, hi, krem);
     if (lo != hi) {
       if (tid == 0) sh.ncand = 0;
       __syncthreads();
@@ -272,11 +276,11 @@ __device__ uint32_t block_topk_regs(const uint32_t (&key)[KPT], int k, EmitFn em
       const uint32_t nc = sh.ncand;
       if (nc <= (uint32_t)kCandCap) {
         auto list = [&](auto&& f) {
-          for (uint32_t i = tid; i < nc; i += blockDim.x) f(sh.cand[i]);
+          for (uint32_t i = tid; i < nc; i += NT) f(sh.cand[i]);
         };
-        while (lo != hi) select_pass(list, sh.t.sel, lo, hi, krem);
+        while (lo != hi) select_pass<NT>(list, sh.t.sel, lo, hi, krem);
       } else {
-        while (lo != hi) select_pass(regs, sh.t.sel, lo, hi, krem);
+        while (lo != hi) select_pass<NT>(regs, sh.t.sel, lo, hi, krem);
       }
     }
   }
@@ -326,7 +330,7 @@ __device__ __forceinline__ void load_keys(const float* row, int n, bool vec, uin
   }
 }
 
-template <int KPT>
+template <int NT, int KPT>
 __device__ void topk_chunk(const TopkParams& P, TopkRegShared& sh) {
   const int q = blockIdx.y;
   const int c = blockIdx.x;
@@ -354,13 +358,13 @@ __device__ void topk_chunk(const TopkParams& P, TopkRegShared& sh) {
   load_keys<KPT>(row, n, vec, key);
   const int p0 = lo + (int)threadIdx.x * KPT;
   if (nchunks <= 1) {
-    const uint32_t cnt = block_topk_regs<KPT>(key, P.topk, [&](uint32_t pos, int r) { out[pos] = p0 + r; }, sh);
+    const uint32_t cnt = block_topk_regs<NT, KPT>(key, P.topk, [&](uint32_t pos, int r) { out[pos] = p0 + r; }, sh);
     for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
   } else {
     const long long cb = ((long long)q * P.max_chunks + c) * P.topk;
     uint32_t* ck = P.cand_key + cb;
     int32_t* ci = P.cand_idx + cb;
-    const uint32_t cnt = block_topk_regs<KPT>(key, P.topk, [&](uint32_t pos, int r) {
+    const uint32_t cnt = block_topk_regs<NT, KPT>(key, P.topk, [&](uint32_t pos, int r) {
       ck[pos] = key[r];
       ci[pos] = p0 + r;
     }, sh);
@@ -377,8 +381,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
   __shared__ TopkRegShared sh;
   pdl_wait();
   pdl_trigger();
-  if (P.max_entries <= 8 * kTopkThreads) topk_chunk<8>(P, sh);  // rows of <= 8192 entries: 8 keys per thread
-  else topk_chunk<kTopkChunk / kTopkThreads>(P, sh);
+  // Rows of <= kTopkShortRow entries hold 8 keys per thread, chunks of kTopkChunk entries 16.
+  if (P.max_entries <= kTopkShortRow) topk_chunk<kTopkShortThreads, kTopkShortRow / kTopkShortThreads>(P, sh);
+  else topk_chunk<kTopkThreads, kTopkChunk / kTopkThreads>(P, sh);
 }
 
 // One CTA per query with more than one chunk: top-k over the union of the chunks' lists. The
