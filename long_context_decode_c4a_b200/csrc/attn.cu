@@ -10,22 +10,29 @@
 //   l_j = scale * q_h . c_j,  m = max(max_j l_j, sink_h),
 //   o_h = sum_j e^(l_j - m) c_j / (sum_j e^(l_j - m) + e^(sink_h - m)),  then rotate o_h[448:] by -t.
 //
-// Layout of the work: two CTAs per query; CTA c accumulates dims [256c, 256c+256) of O. Both
-// gather the full candidate rows (the second read of a row is served by L2) and compute the full
-// scores S = Q K^T (M = 128 heads, N = 32 candidates per tile, K = 512), so they need no
-// communication: each runs the same online softmax on its own copy of S. TMEM's 512 columns hold
-// Q[:, 0:256] as bf16 pairs (the A operand of the TS-MMA for dims 0..255; dims 256..511 come from
-// shared memory), four 32-column score tiles, and O[:, half] (256 columns). With four score
-// tiles the MMA warp runs up to four tiles ahead of the softmax.
-//   SMEM: Q[:, 256:512] (64 KB, 128B-swizzled K-major, TMA); four 32 KB stages of 32 candidate
-//     rows (8 blocks of 64 dims in the 128B-swizzled layout that serves S as a K-major B operand
-//     and PV as an MN-major B operand; Q[:, 0:256] passes through stages 2-3 on its way into
-//     TMEM); the candidate list.
-//   Warps: 0..3 build the candidate list and gather rows with coalesced 16-byte cp.async (then
-//     share the epilogue); 4 and 5 issue the score MMAs of even and odd tiles (one thread issues a
-//     tcgen05.mma only every ~50 cycles, so two issuers keep the tensor pipe fed); 6 issues the PV
-//     MMAs in tile order (and owns TMEM); 7..10 run the softmax (thread = head = TMEM lane) and the
-//     epilogue.
+// Layout of the work: a cluster of two CTAs per query; CTA c owns dims [256c, 256c+256). Each CTA
+// gathers only its half of every candidate row (an SM gathers scattered rows at a fixed rate, so
+// halving the bytes each CTA gathers halves the time this kernel is bound by), computes the
+// partial scores S_c = Q[:, half] K[:, half]^T (M = 128 heads, N = 32 candidates per tile,
+// K = 256) and sends them to the other CTA through distributed shared memory; both add
+// S_0 + S_1 (the same sum in both, fp addition being commutative), run the same online softmax,
+// and accumulate O[:, half] += P V[:, half].
+//   TMEM (512 columns): [0,128) Q[:, half] as bf16 pairs (A operand of the score TS-MMAs);
+//     [128,256) four 32-column score tiles (partial scores, then P_hi in columns [0,16) and P_lo
+//     in [16,32)); [256,512) O[:, half].
+//   SMEM: eight 16 KB stages of 32 half-rows (4 blocks of 64 dims in the 128B-swizzled layout that
+//     serves S as a K-major B operand and PV as an MN-major B operand); two 16 KB outgoing and two
+//     16 KB incoming exchange buffers (together they first stage Q[:, half] on its way into TMEM);
+//     the candidate list.
+//   Warps: 0..3 build the candidate list and gather half-rows with coalesced 16-byte cp.async,
+//     announcing each tile as soon as it lands; 4 and 5 issue the score MMAs of even and odd tiles
+//     (one thread issues a tcgen05.mma only every ~50 cycles); 6 issues the PV MMAs in tile order
+//     (and owns TMEM); 7..10 send the partial scores of their 32 heads (one 4 KB bulk copy per warp
+//     and tile, into the same quadrant's rows of the other CTA's incoming buffer); 11..14 add the
+//     incoming partial scores to their own and run the softmax. A sender and a softmax warp of the
+//     same TMEM lane quadrant trade with the two warps of that quadrant in the other CTA, with
+//     barriers of their own, so the four quadrants run independently; sending tile j+1 overlaps
+//     receiving tile j. Warps 7..14 own one head (TMEM lane) per thread and share the epilogue.
 // Precision: P = P_hi + P_lo with both parts in bf16 (about 16 significant bits), accumulated by two
 // PV MMAs; a single bf16 P (8 bits) leaves errors near 1% of the output RMS on short candidate sets.
 // Online softmax in the log2 domain; the running max starts at the sink; O is rescaled only when a
@@ -47,25 +54,33 @@ constexpr uint32_t kRowMask = 0x3FFFFFFFu;
 constexpr int kProducers = 128;               // warps 0..3
 constexpr int kQkWarp0 = 4;                   // warps 4, 5: score MMAs of even / odd tiles
 constexpr int kPvWarp = 6;                    // PV MMAs; owns TMEM
-constexpr int kSoftWarp0 = 7;                 // warps 7..10
-constexpr int kSoftThreads = 128;
+constexpr int kSendWarp0 = 7;                 // warps 7..10: send partial scores
+constexpr int kSoftWarp0 = 11;                // warps 11..14: softmax
+constexpr int kRoleThreads = 128;
 constexpr int kTile = 32;                     // candidates per tile
-constexpr int kStages = 4;
+constexpr int kStages = 8;
 constexpr int kSBufs = 4;                     // score tiles in TMEM
-constexpr size_t kQhiBytes = 64 * 1024;       // Q[:, 256:512]
-constexpr size_t kStageBytes = 32 * 1024;     // 32 rows x 512 dims of bf16
+constexpr uint32_t kStageBytes = 16 * 1024;   // 32 rows x 256 dims of bf16
 constexpr uint32_t kBlockBytes = 4096;        // one 64-dim block of a stage: [32 rows][128 B]
+constexpr uint32_t kXBytes = 16 * 1024;       // 128 heads x 32 fp32 partial scores
+constexpr int kXBufs = 2;                     // exchange buffers each way
 
 static_assert(kAttnThreads == 32 * (kSoftWarp0 + 4), "warp roles");
 static_assert(kAttnMaxCands % kTile == 0, "candidate capacity");
-
-static_assert(kStages == kSBufs, "tile j uses stage and score tile j % kStages");
+static_assert(kXBufs >= 2 && kXBufs <= kSBufs, "a tile is sent at most kSBufs - 1 tiles ahead");
+static_assert(kXBufs * 2 * kXBytes >= 64 * 1024, "Q[:, half] is staged over the exchange buffers");
 
 struct AttnSmem {
   uint64_t q_full, q_done, list_ready;
-  uint64_t kv_full[kStages];
-  uint64_t buf_free[kStages];         // PV(j) completed: stage and score tile j % kStages are free
-  uint64_t s_full[kSBufs], p_full[kSBufs], o_done[2];
+  uint64_t kv_full[kStages], buf_free[kStages];  // buf_free: PV(j) completed, stage j % kStages free
+  uint64_t s_full[kSBufs], p_full[kSBufs];
+  uint64_t s_free[kSBufs];            // PV(j) completed: score tile j % kSBufs is free, O holds PV(0..j)
+  // Per TMEM lane quadrant q (32 heads): the exchange warp of quadrant q trades its 4 KB of each
+  // tile with the other CTA's exchange warp of quadrant q, and hands the summed scores to the
+  // softmax warp of quadrant q.
+  uint64_t x_sent[kSBufs][4];         // the sender read the partial scores of tile j (score tile j % kSBufs)
+  uint64_t x_full[kXBufs][4];         // incoming 4 KB landed (bulk copy from the other CTA)
+  uint64_t x_empty[kXBufs][4];        // the other CTA consumed the 4 KB this warp sent last
   uint64_t epi;                       // the softmax warps published 1/l
   uint64_t drain[3];
   uint32_t tmem_base;
@@ -93,8 +108,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Byte offset of 16-byte chunk k (0..7) of head row h in a 16 KB exchange buffer (rows of 128
+// bytes); the XOR spreads a quarter-warp's accesses over all banks.
+__device__ __forceinline__ uint32_t xoff(uint32_t h, uint32_t k) { return h * 128u + ((k ^ (h & 7u)) << 4); }
 
 // Exclusive prefix sum over the 128 producer threads (named barrier 2).
 __device__ __forceinline__ uint32_t producer_scan(uint32_t v, uint32_t* scan, uint32_t& total) {
@@ -165,18 +182,20 @@ __device__ __forceinline__ void store_rows(const AttnParams& P, const AttnSmem& 
 
 }  // namespace
 
-__global__ void __launch_bounds__(kAttnThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap map_q, AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* q_hi = base;                       // 4 x [128 rows][128 B]
-  uint8_t* stage0 = base + kQhiBytes;         // stage s at stage0 + s * 32 KB: 8 x [32 rows][128 B]
-  uint8_t* q_lo = stage0 + 2 * kStageBytes;   // Q[:, 0:256] staging over stages 2-3: 4 x [128 rows][128 B]
-  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(stage0 + kStages * kStageBytes);
+  uint8_t* stage0 = base;                        // stage s at stage0 + s * 16 KB: 4 x [32 rows][128 B]
+  uint8_t* xin = base + kStages * kStageBytes;   // kXBufs x 16 KB incoming partial scores
+  uint8_t* xout = xin + kXBufs * kXBytes;        // kXBufs x 16 KB outgoing partial scores
+  uint8_t* qbuf = xin;                           // first Q[:, half]: 4 x [128 rows][128 B]
+  AttnSmem& sm = *reinterpret_cast<AttnSmem*>(xout + kXBufs * kXBytes);
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int half = blockIdx.x;                // which 256 dims of O this CTA owns
+  const uint32_t half = cluster_ctarank();    // which 256 dims this CTA owns
+  const uint32_t peer = half ^ 1u;
   const int nq = P.B * P.S;
   const int qi = nq - 1 - (int)blockIdx.y;    // later queries (more candidates) first
   const int b = qi / P.S;
@@ -185,7 +204,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_done, kSoftThreads);
+    mbar_init(&sm.q_done, 2 * kRoleThreads);
     mbar_init(&sm.list_ready, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.kv_full[i], kProducers);
@@ -193,11 +212,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.p_full[i], kSoftThreads);
+      for (int q = 0; q < 4; ++q) mbar_init(&sm.x_sent[i][q], 32);
+      mbar_init(&sm.p_full[i], kRoleThreads);
+      mbar_init(&sm.s_free[i], 1);
     }
-    mbar_init(&sm.o_done[0], 1);
-    mbar_init(&sm.o_done[1], 1);
-    mbar_init(&sm.epi, kSoftThreads);
+    for (int i = 0; i < kXBufs; ++i) {
+      for (int q = 0; q < 4; ++q) {
+        mbar_init(&sm.x_full[i][q], 1);
+        mbar_init(&sm.x_empty[i][q], 1);
+      }
+    }
+    mbar_init(&sm.epi, kRoleThreads);
     for (int i = 0; i < 3; ++i) mbar_init(&sm.drain[i], 1);
     sm.abort_flag = 0;
     sm.bad = 0;
@@ -208,7 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // the barriers of both CTAs are initialised before any remote access
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   pdl_wait();
@@ -217,15 +242,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) trace_time(status, 0);
 
   if (warp < kProducers / 32) {
-    // ------------------------------------------------------------ Q loads, candidate list, gathers
+    // ------------------------------------------------------------ Q load, candidate list, gathers
     const int pt = threadIdx.x;  // 0..127
-    const int quad = warp & 3;
-    const int h = quad * 32 + lane;
     if (pt == 0) {
       const int row0 = qi * P.H;
-      mbar_arrive_expect_tx(&sm.q_full, 8u * 16384u);
-      for (int k = 0; k < 4; ++k) tma_load_2d(q_hi + k * 16384, &map_q, 256 + 64 * k, row0, &sm.q_full);
-      for (int k = 0; k < 4; ++k) tma_load_2d(q_lo + k * 16384, &map_q, 64 * k, row0, &sm.q_full);
+      mbar_arrive_expect_tx(&sm.q_full, 4u * 16384u);
+      for (int k = 0; k < 4; ++k) tma_load_2d(qbuf + k * 16384, &map_q, 256 * (int)half + 64 * k, row0, &sm.q_full);
     }
     // Candidate list: window rows, then the compressed entries, padded to tiles of 32.
     const long long ring_row0 = (long long)b * P.ring_rows;
@@ -290,43 +312,34 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       trace_time(status, 1);
     }
 
-    // Gathers: tile j -> stage j % kStages. Thread pt copies the 16-byte chunks pt, pt+128, ... of
-    // the tile (32 rows x 64 chunks): a warp covers 512 contiguous bytes of one row per
-    // instruction. The loop issues the next tile whenever its stage is free and otherwise waits
-    // for its oldest tile in flight and announces it (kv_full), so tiles are announced as soon as
-    // they land while up to kStages tiles are in flight. Each thread runs the loop on its own
-    // (its decisions may differ from other threads'); every thread arrives once per tile. Stages
-    // 2 and 3 first hold Q[:, 0:256] until the softmax warps moved it into TMEM (q_done).
-    const char* ring_base = reinterpret_cast<const char*>(P.ring);
-    const char* cache_base = reinterpret_cast<const char*>(P.cache);
+    // Gathers: tile j -> stage j % kStages, this CTA's 512 bytes of each of its 32 rows. Thread pt
+    // copies the 16-byte chunks pt, pt+128, ... of the tile (32 rows x 32 chunks): a warp covers
+    // the 512 contiguous bytes of one row per instruction. The loop issues the next tile whenever
+    // its stage is free and otherwise waits for its oldest tile in flight and announces it
+    // (kv_full), so tiles are announced as soon as they land while up to kStages tiles are in
+    // flight. Each thread runs the loop on its own (its decisions may differ from other threads');
+    // every thread arrives once per tile.
+    const char* ring_base = reinterpret_cast<const char*>(P.ring) + 512 * half;
+    const char* cache_base = reinterpret_cast<const char*>(P.cache) + 512 * half;
     int next = 0, ann = 0;
-    bool ok = true;
     while (ann < J) {
       bool issue = next < J;
-      if (issue && next >= 2 && next < kStages) {
-        if (next > ann) {
-          issue = mbar_test(smem_u32(&sm.q_done), 0);
-        } else if (!mbar_wait(&sm.q_done, 0, abort_flag, status, 101)) {
-          ok = false;
-          break;
-        }
-      } else if (issue && next >= kStages) {
+      if (issue && next >= kStages) {
         uint64_t* empty = &sm.buf_free[next % kStages];
         const uint32_t par = (uint32_t)((next / kStages - 1) & 1);
         if (next > ann) {
           issue = mbar_test(smem_u32(empty), par);
         } else if (!mbar_wait(empty, par, abort_flag, status, 102)) {
-          ok = false;
           break;
         }
       }
       if (issue) {
         const uint32_t st = smem_u32(stage0 + (size_t)(next % kStages) * kStageBytes);
-#pragma unroll 8
-        for (int i = 0; i < 16; ++i) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
           const int c = pt + kProducers * i;  // chunk of the tile
-          const int r = c >> 6;               // candidate row 0..31
-          const int w = c & 63;               // chunk within the row
+          const int r = c >> 5;               // candidate row 0..31
+          const int w = c & 31;               // chunk within the half-row
           const uint32_t e = sm.list[next * kTile + r];
           const char* src = ((e & kFromCache) ? cache_base : ring_base) + (size_t)(e & kRowMask) * 1024 + w * 16;
           cp_async_16(st + (w >> 3) * kBlockBytes + sw128_offset(r, w & 7), src);
@@ -339,7 +352,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         case 1: cp_async_wait<0>(); break;
         case 2: cp_async_wait<1>(); break;
         case 3: cp_async_wait<2>(); break;
-        default: cp_async_wait<3>(); break;
+        case 4: cp_async_wait<3>(); break;
+        case 5: cp_async_wait<4>(); break;
+        case 6: cp_async_wait<5>(); break;
+        case 7: cp_async_wait<6>(); break;
+        default: cp_async_wait<7>(); break;
       }
       fence_proxy_async_smem();
       mbar_arrive(&sm.kv_full[ann % kStages]);
@@ -347,46 +364,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ++ann;
     }
     cp_async_wait<0>();  // after an abort: let the copies land before teardown
-    // Epilogue share: O columns [128, 256) of this warp's rows, once the softmax published 1/l.
-    const bool fin =
-        __all_sync(0xffffffffu, ok && ann == J && J > 0 && mbar_wait(&sm.epi, 0, abort_flag, status, 103));
-    if (fin) {
-      tc_fence_after();
-      store_rows(P, sm, tmem + ((uint32_t)(quad * 32) << 16) + 256, 128, half, (long long)qi * P.H + h, h,
-                 sm.inv_l[h]);
-    }
   } else if (warp < kPvWarp) {
     // ------------------------------------------------------------ score MMAs: tiles j = w, w+2, ...
     if (lane == 0) {
       const int w = warp - kQkWarp0;  // 0: even tiles, 1: odd tiles
-      bool ok = mbar_wait(&sm.q_full, 0, abort_flag, status, 111) &&
-                mbar_wait(&sm.q_done, 0, abort_flag, status, 112) &&
+      bool ok = mbar_wait(&sm.q_done, 0, abort_flag, status, 112) &&
                 mbar_wait(&sm.list_ready, 0, abort_flag, status, 113);
       const int J = ok ? sm.n_tiles : 0;
       const uint32_t idesc_qk = idesc_bf16_f32(128, kTile, 0, 0);
-      const uint32_t qhi = smem_u32(q_hi);
       for (int j = w; j < J; j += 2) {
-        const int s = j % kStages;
-        // Score tile s is rewritten only once PV(j - kStages), which read its P, has completed.
-        if (j >= kStages && !mbar_wait(&sm.buf_free[s], (uint32_t)((j / kStages - 1) & 1), abort_flag, status, 117))
+        const int s = j % kStages, sb = j % kSBufs;
+        // Score tile sb is rewritten only once PV(j - kSBufs), which read its P, has completed.
+        if (j >= kSBufs && !mbar_wait(&sm.s_free[sb], (uint32_t)((j / kSBufs - 1) & 1), abort_flag, status, 117))
           break;
         if (!mbar_wait(&sm.kv_full[s], (uint32_t)((j / kStages) & 1), abort_flag, status, 114)) break;
         tc_fence_after();
         if (j < 60) trace_time(status, 64 + j);
         const uint32_t kbase = smem_u32(stage0 + (size_t)s * kStageBytes);
-        const uint32_t d_s = tmem + 128 + kTile * s;
+        const uint32_t d_s = tmem + 128 + kTile * sb;
 #pragma unroll
-        for (int ks = 0; ks < 16; ++ks) {  // dims 0..255: A = Q from TMEM
+        for (int ks = 0; ks < 16; ++ks) {  // this CTA's 256 dims: A = Q[:, half] from TMEM
           const uint64_t bdesc = smem_desc_sw128(kbase + (ks >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024);
           mma_ts(d_s, tmem + 8 * ks, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
         }
-#pragma unroll
-        for (int ks = 16; ks < 32; ++ks) {  // dims 256..511: A = Q from smem
-          const uint64_t adesc = smem_desc_sw128(qhi + ((ks - 16) >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(kbase + (ks >> 2) * kBlockBytes + (ks & 3) * 32, 16, 1024);
-          mma_ss(d_s, adesc, bdesc, idesc_qk, 1u);
-        }
-        mma_commit(&sm.s_full[s]);
+        mma_commit(&sm.s_full[sb]);
       }
       // Every MMA issued above completes on its own; wait for them before TMEM is released.
       mma_commit(&sm.drain[w]);
@@ -402,8 +403,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int sb = j % kSBufs;
         if (!mbar_wait(&sm.p_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 115)) break;
         tc_fence_after();
-        const uint32_t vbase =
-            smem_u32(stage0 + (size_t)(j % kStages) * kStageBytes) + (uint32_t)(4 * half) * kBlockBytes;
+        const uint32_t vbase = smem_u32(stage0 + (size_t)(j % kStages) * kStageBytes);
         const uint32_t pcol = tmem + 128 + kTile * sb;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {  // P_hi, then P_lo
@@ -413,28 +413,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mma_ts(tmem + 256, pcol + 16 * part + 8 * ks, bdesc, idesc_pv, (j > 0 || part > 0 || ks > 0) ? 1u : 0u);
           }
         }
-        mma_commit(&sm.o_done[j & 1]);
         mma_commit(&sm.buf_free[j % kStages]);
+        mma_commit(&sm.s_free[sb]);
         if (j < 60) trace_time(status, 192 + j);
       }
       mma_commit(&sm.drain[2]);
       mbar_wait_drain(&sm.drain[2], 0, status, 119);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 5..8), epilogue
+    // ------------------------------------------------------------ senders (7..10), softmax (11..14)
+    const bool sender = warp < kSoftWarp0;
     const int quad = warp & 3;             // TMEM lane quadrant
     const int h = quad * 32 + lane;        // head = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const int et = threadIdx.x - kSoftWarp0 * 32;
-    // Q[:, 0:256] -> TMEM columns [0, 128).
+    const int rt = threadIdx.x - (sender ? kSendWarp0 : kSoftWarp0) * 32;  // 0..127 within the role
+    // Q[:, half] -> TMEM columns [0, 128): blocks 0-1 by the senders, 2-3 by the softmax warps.
     bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag, status, 121));
     if (ok) {
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
+      for (int kk = 0; kk < 2; ++kk) {
+        const int kb = (sender ? 0 : 2) + kk;
         uint32_t r[32];
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
-          const uint4 v = *reinterpret_cast<const uint4*>(q_lo + kb * 16384 + sw128_offset(h, ch));
+          const uint4 v = *reinterpret_cast<const uint4*>(qbuf + kb * 16384 + sw128_offset(h, ch));
           r[4 * ch + 0] = v.x;
           r[4 * ch + 1] = v.y;
           r[4 * ch + 2] = v.z;
@@ -448,112 +450,206 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_arrive(&sm.q_done);
     // Inverse-RoPE table for position t.
     const int npairs = P.rope_dim / 2;
-    if (et < npairs) {
+    if (!sender && rt < npairs) {
       float cs, sn;
-      rope_cos_sin(t, P.inv_freq[et], &cs, &sn);
-      sm.rope_cs[et][0] = cs;
-      sm.rope_cs[et][1] = -sn;
+      rope_cos_sin(t, P.inv_freq[rt], &cs, &sn);
+      sm.rope_cs[rt][0] = cs;
+      sm.rope_cs[rt][1] = -sn;
     }
-    named_bar_sync(1, kSoftThreads);
+    named_bar_sync(1, 2 * kRoleThreads);   // the Q staging area is no longer read
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&sm.list_ready, 0, abort_flag, status, 122));
     const int J = ok ? sm.n_tiles : 0;
-    const float sl = (h < P.H) ? P.sink[h] * 1.4426950408889634f : 0.f;
-    float m_used = sl;  // running max in log2 units (starts at the sink)
-    float l = 1.f;      // running denominator; the sink contributes exp2(sl - m_used) = 1
+    // Tile j travels through exchange buffer c = j % kXBufs; phase (j / kXBufs) & 1 of x_full /
+    // x_empty [c][quad] belongs to it. The sender and softmax warps of quadrant quad own the 4 KB
+    // of its 32 heads (rows [32 quad, 32 quad + 32) of every exchange buffer) and trade them with
+    // the warps of the same quadrant in the other CTA.
+    const uint32_t qoff = (uint32_t)quad * (kXBytes / 4);
+    const uint32_t xempty_peer = mapa_shared(smem_u32(&sm.x_empty[0][quad]), peer);
     int j = 0;
-    for (; j < J; ++j) {
-      const int sb = j % kSBufs;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 123)))
-        break;
-      if (et == 0 && j < 60) trace_time(status, 500 + j);
-      tc_fence_after();
-      const uint32_t sa = tmem + lane_addr + 128 + kTile * sb;
-      uint32_t v[32];
-      tmem_ld32(sa, v);
-      tmem_wait_ld();
-      const uint32_t mk = sm.mask[j];
-      float x[32];
-      float mt = -CUDART_INF_F;
-      if (mk == 0xFFFFFFFFu) {  // a full tile (the common case): no padding to mask
+    if (sender) {
+      const uint32_t xin_peer = mapa_shared(smem_u32(xin), peer) + qoff;
+      const uint32_t xfull_peer = mapa_shared(smem_u32(&sm.x_full[0][quad]), peer);
+      for (; j < J; ++j) {
+        const int c = j % kXBufs, sb = j % kSBufs;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 123)))
+          break;
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_addr + 128 + kTile * sb, v);
+        tmem_wait_ld();
+        // The partial scores are read: the softmax warp may overwrite the score tile with P.
+        tc_fence_before();
+        mbar_arrive(&sm.x_sent[sb][quad]);
+        // The other CTA consumed tile j - kXBufs: its incoming buffer c and this CTA's outgoing
+        // buffer c (read by that copy) are free.
+        if (!__all_sync(0xffffffffu, mbar_wait_cluster(&sm.x_empty[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag,
+                                                        status, 126)))
+          break;
+        uint8_t* xo = xout + c * kXBytes;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(v[c]) * P.scale_log2;
-          mt = fmaxf(mt, x[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = ((mk >> c) & 1u) ? __uint_as_float(v[c]) * P.scale_log2 : -CUDART_INF_F;
-          mt = fmaxf(mt, x[c]);
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<uint4*>(xo + xoff(h, i)) = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          bulk_copy_to_cluster(xin_peer + c * kXBytes, smem_u32(xo) + qoff, kXBytes / 4, xfull_peer + 32 * c);
+          if (rt == 0 && j < 60) trace_time(status, 300 + j);
         }
       }
-      // Lazy rescale: only when this tile raises the row max by more than 2^8. The TMEM accesses
-      // are warp-collective, so the whole warp takes the branch if any lane needs it (lanes that do
-      // not need it scale by 1).
-      const bool need = mt > m_used + 8.f;
-      const float alpha = need ? exp2f(m_used - mt) : 1.f;
-      if (__any_sync(0xffffffffu, need)) {
-        if (j > 0) {
-          // O holds PV(0..j-1): wait for PV(j-1), then scale the rows of this warp.
-          const bool okw = mbar_wait(&sm.o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort_flag, status, 124);
-          if (!__all_sync(0xffffffffu, okw)) break;
-          tc_fence_after();
-#pragma unroll 1
-          for (int cc = 0; cc < 8; ++cc) {
-            uint32_t o[32];
-            const uint32_t oa = tmem + lane_addr + 256 + 32 * cc;
-            tmem_ld32(oa, o);
-            tmem_wait_ld();
+    } else {
+      // Every incoming buffer is free: arm them, then let the other CTA send.
+      if (lane == 0)
+        for (int c = 0; c < kXBufs; ++c) {
+          mbar_arrive_expect_tx(&sm.x_full[c][quad], kXBytes / 4);
+          mbar_arrive_remote_relaxed(xempty_peer + 32 * c);
+        }
+      const float sl = (h < P.H) ? P.sink[h] * 1.4426950408889634f : 0.f;
+      float m_used = sl;  // running max in log2 units (starts at the sink)
+      float l = 1.f;      // running denominator; the sink contributes exp2(sl - m_used) = 1
+      // s_free[i % kSBufs] completes once per PV(i). A parity wait for PV(i) is unambiguous while
+      // PV(i - kSBufs) has been observed and PV(i + kSBufs) cannot have completed, so PV
+      // completions are observed in order: PV(j - kSBufs) at tile j (it completed before the score
+      // MMAs of tile j were issued, so this never blocks; PV(j) is not issued yet), which makes
+      // PV(j - 1) safe to wait for before a rescale, and PV(J - 1) before the epilogue.
+      int pv_seen = 0;  // PV(0 .. pv_seen-1) observed complete
+      auto observe_pv = [&](int upto) -> bool {  // observe PV(pv_seen .. upto-1)
+        for (; pv_seen < upto; ++pv_seen)
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_free[pv_seen % kSBufs], (uint32_t)((pv_seen / kSBufs) & 1),
+                                                 abort_flag, status, 124)))
+            return false;
+        return true;
+      };
+      for (; j < J; ++j) {
+        const int c = j % kXBufs, sb = j % kSBufs;
+        const uint32_t sa = tmem + lane_addr + 128 + kTile * sb;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 128)))
+          break;
+        if (!observe_pv(j - kSBufs + 1)) break;
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld32(sa, v);
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_full[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag, status, 127)))
+          break;
+        if (rt == 0 && j < 60) trace_time(status, 400 + j);
+        tmem_wait_ld();
+        // S = S_0 + S_1 (the same sum in both CTAs), scaled to log2 units; padding -> -inf.
+        const uint8_t* xi = xin + c * kXBytes;
+        const uint32_t mk = sm.mask[j];
+        float x[32];
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(oa, o);
+        for (int i = 0; i < 8; ++i) {
+          const uint4 o = *reinterpret_cast<const uint4*>(xi + xoff(h, i));
+          const float ov[4] = {__uint_as_float(o.x), __uint_as_float(o.y), __uint_as_float(o.z), __uint_as_float(o.w)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int cc = 4 * i + e;
+            const float sc = (__uint_as_float(v[cc]) + ov[e]) * P.scale_log2;
+            x[cc] = ((mk >> cc) & 1u) ? sc : -CUDART_INF_F;
           }
-          tmem_wait_st();
         }
-        if (need) {
-          l *= alpha;
-          m_used = mt;
-        }
-      }
-      // P = P_hi + P_lo, both bf16: P_hi in columns [0,16) of the tile, P_lo in [16,32).
-      uint32_t phi[16], plo[16];
-      float rs = 0.f;
+        float mt;
+        {
+          float r[16];
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const float p0 = ex2_approx(x[2 * q] - m_used);
-        const float p1 = ex2_approx(x[2 * q + 1] - m_used);
-        phi[q] = pack_bf16(p0, p1);
-        plo[q] = pack_bf16(p0 - bf16_lo(phi[q]), p1 - bf16_hi(phi[q]));
-        rs += p0 + p1;
+          for (int e = 0; e < 16; ++e) r[e] = fmaxf(x[e], x[e + 16]);
+#pragma unroll
+          for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+            for (int e = 0; e < w; ++e) r[e] = fmaxf(r[e], r[e + w]);
+          mt = r[0];
+        }
+        // mt depends on every value the warp loaded from the buffer (and a warp's loads complete
+        // together), so once it is formed the buffer can be armed for tile j + kXBufs and released
+        // to the other CTA.
+        asm volatile("" ::"f"(mt) : "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sm.x_full[c][quad], kXBytes / 4);
+          mbar_arrive_remote_relaxed(xempty_peer + 32 * c);
+        }
+        if (rt == 0 && j < 60) trace_time(status, 500 + j);
+        // Lazy rescale: only when this tile raises the row max by more than 2^8. The TMEM accesses
+        // are warp-collective, so the whole warp takes the branch if any lane needs it (lanes that do
+        // not need it scale by 1).
+        const bool need = mt > m_used + 8.f;
+        const float alpha = need ? exp2f(m_used - mt) : 1.f;
+        if (__any_sync(0xffffffffu, need)) {
+          if (j > 0) {
+            // O holds PV(0..j-1): wait for PV(j-1), then scale the rows of this warp.
+            if (!observe_pv(j)) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < 8; ++cc) {
+              uint32_t o[32];
+              const uint32_t oa = tmem + lane_addr + 256 + 32 * cc;
+              tmem_ld32(oa, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(oa, o);
+            }
+            tmem_wait_st();
+          }
+          if (need) {
+            l *= alpha;
+            m_used = mt;
+          }
+        }
+        // P = P_hi + P_lo, both bf16: P_hi in columns [0,16) of the tile, P_lo in [16,32). P_hi is p
+        // truncated to bf16 (the high half of its bits); P_lo = p - P_hi is exact in fp32 and is
+        // rounded to bf16, so P_hi + P_lo is within 2^-16 of p relative.
+        uint32_t phi[16], plo[16];
+        float ps[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float p0 = ex2_approx(x[2 * q] - m_used);
+          const float p1 = ex2_approx(x[2 * q + 1] - m_used);
+          const uint32_t u0 = __float_as_uint(p0), u1 = __float_as_uint(p1);
+          phi[q] = __byte_perm(u0, u1, 0x7632);
+          plo[q] = pack_bf16(p0 - __uint_as_float(u0 & 0xFFFF0000u), p1 - __uint_as_float(u1 & 0xFFFF0000u));
+          ps[q] = p0 + p1;
+        }
+#pragma unroll
+        for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) ps[e] += ps[e + w];
+        l += ps[0];
+        // The sender has read this tile's partial scores before P overwrites them.
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_sent[sb][quad], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 129)))
+          break;
+        tc_fence_after();
+        tmem_st16(sa, phi);
+        tmem_st16(sa + 16, plo);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[sb]);
+        if (rt == 0 && j < 60) trace_time(status, 128 + j);
       }
-      l += rs;
-      tmem_st16(sa, phi);
-      tmem_st16(sa + 16, plo);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sm.p_full[sb]);
-      if (et == 0 && j < 60) trace_time(status, 128 + j);
+      if (j == J && !observe_pv(J)) j = -1;
+      sm.inv_l[h] = 1.f / l;
     }
-    // Epilogue: this warp's rows, O columns [0, 128); the producer warps take [128, 256).
-    const bool fin = __all_sync(0xffffffffu, j == J && J > 0 &&
-                                                 mbar_wait(&sm.o_done[(J - 1) & 1], (uint32_t)(((J - 1) >> 1) & 1),
-                                                           abort_flag, status, 125));
-    const float inv = 1.f / l;
-    sm.inv_l[h] = inv;
-    mbar_arrive(&sm.epi);
+    // Epilogue: O / l, inverse RoPE on the rotated dims, store. The softmax warps take O columns
+    // [0, 128) of their rows, the senders [128, 256).
+    bool fin;
+    if (sender) {
+      fin = __all_sync(0xffffffffu, j == J && J > 0 && mbar_wait(&sm.epi, 0, abort_flag, status, 125));
+    } else {
+      fin = __all_sync(0xffffffffu, j == J && J > 0);  // every PV observed complete
+      mbar_arrive(&sm.epi);
+    }
     if (fin) {
       tc_fence_after();
-      store_rows(P, sm, tmem + lane_addr + 256, 0, half, (long long)qi * P.H + h, h, inv);
+      store_rows(P, sm, tmem + lane_addr + 256, sender ? 128 : 0, (int)half, (long long)qi * P.H + h, h, sm.inv_l[h]);
     }
   }
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // no remote access into this CTA's shared memory after this point
   tc_fence_after();
   if (threadIdx.x == 0) trace_time(status, 255);
   if (warp == kPvWarp) tmem_dealloc(tmem, 512);
 }
 
-size_t attn_smem_bytes() { return 1024 + kQhiBytes + kStages * kStageBytes + sizeof(AttnSmem); }
+size_t attn_smem_bytes() { return 1024 + kStages * kStageBytes + 2 * kXBufs * (size_t)kXBytes + sizeof(AttnSmem); }
 
 }  // namespace csa
