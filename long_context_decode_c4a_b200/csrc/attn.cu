@@ -59,34 +59,41 @@ constexpr int kSoftWarp0 = 11;                // warps 11..14: softmax
 constexpr int kRoleThreads = 128;
 constexpr int kTile = 32;                     // candidates per tile
 constexpr int kStages = 8;
-constexpr int kSBufs = 4;                     // score tiles in TMEM
+constexpr int kSBufs = 2;                     // partial-score tiles in TMEM
 constexpr uint32_t kStageBytes = 16 * 1024;   // 32 rows x 256 dims of bf16
 constexpr uint32_t kBlockBytes = 4096;        // one 64-dim block of a stage: [32 rows][128 B]
 constexpr uint32_t kXBytes = 16 * 1024;       // 128 heads x 32 fp32 partial scores
+constexpr uint32_t kOutRow = 512 + 16;        // bf16 output staging: 256 dims per head row, padded
 constexpr int kXBufs = 2;                     // exchange buffers each way
+constexpr int kPBufs = 2;                     // P tiles in TMEM
 
 static_assert(kAttnThreads == 32 * (kSoftWarp0 + 4), "warp roles");
 static_assert(kAttnMaxCands % kTile == 0, "candidate capacity");
-static_assert(kXBufs >= 2 && kXBufs <= kSBufs, "a tile is sent at most kSBufs - 1 tiles ahead");
+static_assert(kXBufs >= 2, "exchange buffers");
 static_assert(kXBufs * 2 * kXBytes >= 64 * 1024, "Q[:, half] is staged over the exchange buffers");
 
 struct AttnSmem {
   uint64_t q_full, q_done, list_ready;
   uint64_t kv_full[kStages], buf_free[kStages];  // buf_free: PV(j) completed, stage j % kStages free
-  uint64_t s_full[kSBufs], p_full[kSBufs];
-  uint64_t s_free[kSBufs];            // PV(j) completed: score tile j % kSBufs is free, O holds PV(0..j)
-  // Per TMEM lane quadrant q (32 heads): the exchange warp of quadrant q trades its 4 KB of each
-  // tile with the other CTA's exchange warp of quadrant q, and hands the summed scores to the
-  // softmax warp of quadrant q.
-  uint64_t x_sent[kSBufs][4];         // the sender read the partial scores of tile j (score tile j % kSBufs)
+  uint64_t s_full[kSBufs];            // score MMAs of tile j done (score tile j % kSBufs)
+  uint64_t s_rd[kSBufs];              // the senders read the partial scores of tile j
+  uint64_t p_full[kPBufs];            // P of tile j stored (P tile j % kPBufs)
+  uint64_t p_free[kPBufs];            // PV(j) completed: P tile j % kPBufs is free, O holds PV(0..j)
+  // Per TMEM lane quadrant q (32 heads): the sender warp of quadrant q stages its 4 KB of each
+  // tile in the outgoing buffer and copies it to the same rows of the other CTA's incoming buffer;
+  // the softmax warp of quadrant q reads its own 4 KB from the outgoing buffer and the other CTA's
+  // from the incoming buffer.
   uint64_t x_full[kXBufs][4];         // incoming 4 KB landed (bulk copy from the other CTA)
   uint64_t x_empty[kXBufs][4];        // the other CTA consumed the 4 KB this warp sent last
+  uint64_t x_staged[kXBufs][4];       // this CTA's 4 KB is staged in the outgoing buffer
+  uint64_t x_own[kXBufs][4];          // this CTA's softmax warp read its staged 4 KB
   uint64_t epi;                       // the softmax warps published 1/l
   uint64_t drain[3];
   uint32_t tmem_base;
   int abort_flag;
   int n_tiles;
   int bad;
+  int epi_bad;                        // some epilogue warp lacks a complete O
   uint32_t scan[kProducers / 32];
   float rope_cs[kMaxRopePairs][2];
   float inv_l[128];
@@ -136,13 +143,15 @@ __device__ __forceinline__ uint32_t producer_scan(uint32_t v, uint32_t* scan, ui
   return off + inc - v;
 }
 
-// O[:, half] / l for 128 of this CTA's 256 dims of row h (columns [c0, c0+128) of its O), the
-// inverse RoPE on the rotated dims, and the store. Warp-collective (TMEM loads).
-__device__ __forceinline__ void store_rows(const AttnParams& P, const AttnSmem& sm, uint32_t o_taddr, int c0,
-                                           int half, long long orow, int h, float inv) {
+// O[:, half] / l for columns [c0, c0 + 32 nchunks) of this CTA's 256 dims of row h (the global dims
+// [256 half + c0, ...)), with the inverse RoPE on the rotated dims. fp32 output is stored to global
+// memory directly; bf16 output goes to the staging row `srow` (this CTA's 512 bytes of the output
+// row) for one bulk store per row. Warp-collective (TMEM loads).
+__device__ __forceinline__ void finish_rows(const AttnParams& P, const AttnSmem& sm, uint32_t o_taddr, int c0, int nchunks,
+                                            int half, long long orow, int h, float inv, uint8_t* srow) {
   const int rope0 = P.d - P.rope_dim;  // first rotated dim
 #pragma unroll 1
-  for (int cc = 0; cc < 4; ++cc) {
+  for (int cc = 0; cc < nchunks; ++cc) {
     const int lc = c0 + 32 * cc;
     uint32_t o[32];
     tmem_ld32(o_taddr + lc, o);
@@ -164,18 +173,18 @@ __device__ __forceinline__ void store_rows(const AttnParams& P, const AttnSmem& 
         }
       }
     }
-    if (h < P.H) {
-      if (P.out_is_f32) {
+    if (P.out_is_f32) {
+      if (h < P.H) {
         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(P.out) + orow * P.d + col0);
 #pragma unroll
         for (int c = 0; c < 8; ++c) dst[c] = make_float4(y[4 * c], y[4 * c + 1], y[4 * c + 2], y[4 * c + 3]);
-      } else {
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(P.out) + orow * P.d + col0);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          dst[c] = make_uint4(pack_bf16(y[8 * c], y[8 * c + 1]), pack_bf16(y[8 * c + 2], y[8 * c + 3]),
-                              pack_bf16(y[8 * c + 4], y[8 * c + 5]), pack_bf16(y[8 * c + 6], y[8 * c + 7]));
       }
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(srow + 2 * lc);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        dst[c] = make_uint4(pack_bf16(y[8 * c], y[8 * c + 1]), pack_bf16(y[8 * c + 2], y[8 * c + 3]),
+                            pack_bf16(y[8 * c + 4], y[8 * c + 5]), pack_bf16(y[8 * c + 6], y[8 * c + 7]));
     }
   }
 }
@@ -212,20 +221,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     }
     for (int i = 0; i < kSBufs; ++i) {
       mbar_init(&sm.s_full[i], 1);
-      for (int q = 0; q < 4; ++q) mbar_init(&sm.x_sent[i][q], 32);
+      mbar_init(&sm.s_rd[i], kRoleThreads);
+    }
+    for (int i = 0; i < kPBufs; ++i) {
       mbar_init(&sm.p_full[i], kRoleThreads);
-      mbar_init(&sm.s_free[i], 1);
+      mbar_init(&sm.p_free[i], 1);
     }
     for (int i = 0; i < kXBufs; ++i) {
       for (int q = 0; q < 4; ++q) {
         mbar_init(&sm.x_full[i][q], 1);
         mbar_init(&sm.x_empty[i][q], 1);
+        mbar_init(&sm.x_staged[i][q], 1);
+        mbar_init(&sm.x_own[i][q], 1);
       }
     }
     mbar_init(&sm.epi, kRoleThreads);
     for (int i = 0; i < 3; ++i) mbar_init(&sm.drain[i], 1);
     sm.abort_flag = 0;
     sm.bad = 0;
+    sm.epi_bad = 0;
     fence_mbar_init();
   }
   if (warp == kPvWarp) {
@@ -257,6 +271,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     const uint32_t self_slot = (uint32_t)(ring_row0 + (t % P.ring_cap)) & kRowMask;
     for (int k = pt; k < nwin; k += kProducers)
       sm.list[k] = (uint32_t)(ring_row0 + (long long)((p0 + k) % P.ring_cap)) & kRowMask;
+    // Gather of tile `tile` into stage tile % kStages: this CTA's 512 bytes of each of its 32 rows.
+    // Thread pt copies the 16-byte chunks pt, pt+128, ... of the tile (32 rows x 32 chunks): a warp
+    // covers the 512 contiguous bytes of one row per instruction.
+    const char* ring_base = reinterpret_cast<const char*>(P.ring) + 512 * half;
+    const char* cache_base = reinterpret_cast<const char*>(P.cache) + 512 * half;
+    auto issue = [&](int tile) {
+      const uint32_t st = smem_u32(stage0 + (size_t)(tile % kStages) * kStageBytes);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = pt + kProducers * i;  // chunk of the tile
+        const int r = c >> 5;               // candidate row 0..31
+        const int w = c & 31;               // chunk within the half-row
+        const uint32_t e = sm.list[tile * kTile + r];
+        const char* src = ((e & kFromCache) ? cache_base : ring_base) + (size_t)(e & kRowMask) * 1024 + w * 16;
+        cp_async_16(st + (w >> 3) * kBlockBytes + sw128_offset(r, w & 7), src);
+      }
+      cp_async_commit();
+    };
+    // Tiles made only of window rows are known now: their gathers start before the compressed
+    // entries are read.
+    named_bar_sync(2, kProducers);
+    const int w_tiles = min(nwin / kTile, kStages);
+    for (int tile = 0; tile < w_tiles; ++tile) issue(tile);
     const int ecap = min((t + 1) / P.ratio, P.max_entries);
     int n = nwin;
     bool bad = false;
@@ -297,12 +334,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     const int nt = (n + kTile - 1) & ~(kTile - 1);
     for (int k = n + pt; k < nt; k += kProducers) sm.list[k] = self_slot | kInvalid;
     const int J = nt / kTile;
-    named_bar_sync(2, kProducers);
+    // Entries [0, n) are valid, [n, nt) padding.
     for (int j = pt; j < J; j += kProducers) {
-      uint32_t mk = 0;
-      for (int c = 0; c < kTile; ++c)
-        if (!(sm.list[j * kTile + c] & kInvalid)) mk |= 1u << c;
-      sm.mask[j] = mk;
+      const int rem = n - j * kTile;
+      sm.mask[j] = rem >= kTile ? 0xFFFFFFFFu : (rem > 0 ? (1u << rem) - 1u : 0u);
     }
     if (pt == 0) sm.n_tiles = J;
     named_bar_sync(2, kProducers);
@@ -312,39 +347,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       trace_time(status, 1);
     }
 
-    // Gathers: tile j -> stage j % kStages, this CTA's 512 bytes of each of its 32 rows. Thread pt
-    // copies the 16-byte chunks pt, pt+128, ... of the tile (32 rows x 32 chunks): a warp covers
-    // the 512 contiguous bytes of one row per instruction. The loop issues the next tile whenever
-    // its stage is free and otherwise waits for its oldest tile in flight and announces it
-    // (kv_full), so tiles are announced as soon as they land while up to kStages tiles are in
-    // flight. Each thread runs the loop on its own (its decisions may differ from other threads');
-    // every thread arrives once per tile.
-    const char* ring_base = reinterpret_cast<const char*>(P.ring) + 512 * half;
-    const char* cache_base = reinterpret_cast<const char*>(P.cache) + 512 * half;
-    int next = 0, ann = 0;
+    // Gathers: tile j -> stage j % kStages. The loop issues the next tile whenever its stage is free
+    // and otherwise waits for its oldest tile in flight and announces it (kv_full), so tiles are
+    // announced as soon as they land while up to kStages tiles are in flight. Each thread runs the
+    // loop on its own (its decisions may differ from other threads'); every thread arrives once
+    // per tile.
+    int next = w_tiles, ann = 0;
     while (ann < J) {
-      bool issue = next < J;
-      if (issue && next >= kStages) {
+      bool go = next < J;
+      if (go && next >= kStages) {
         uint64_t* empty = &sm.buf_free[next % kStages];
         const uint32_t par = (uint32_t)((next / kStages - 1) & 1);
         if (next > ann) {
-          issue = mbar_test(smem_u32(empty), par);
+          go = mbar_test(smem_u32(empty), par);
         } else if (!mbar_wait(empty, par, abort_flag, status, 102)) {
           break;
         }
       }
-      if (issue) {
-        const uint32_t st = smem_u32(stage0 + (size_t)(next % kStages) * kStageBytes);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int c = pt + kProducers * i;  // chunk of the tile
-          const int r = c >> 5;               // candidate row 0..31
-          const int w = c & 31;               // chunk within the half-row
-          const uint32_t e = sm.list[next * kTile + r];
-          const char* src = ((e & kFromCache) ? cache_base : ring_base) + (size_t)(e & kRowMask) * 1024 + w * 16;
-          cp_async_16(st + (w >> 3) * kBlockBytes + sw128_offset(r, w & 7), src);
-        }
-        cp_async_commit();
+      if (go) {
+        issue(next);
         ++next;
         continue;
       }
@@ -374,8 +395,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       const uint32_t idesc_qk = idesc_bf16_f32(128, kTile, 0, 0);
       for (int j = w; j < J; j += 2) {
         const int s = j % kStages, sb = j % kSBufs;
-        // Score tile sb is rewritten only once PV(j - kSBufs), which read its P, has completed.
-        if (j >= kSBufs && !mbar_wait(&sm.s_free[sb], (uint32_t)((j / kSBufs - 1) & 1), abort_flag, status, 117))
+        // Score tile sb is rewritten only once the senders have loaded tile j - kSBufs.
+        if (j >= kSBufs && !mbar_wait(&sm.s_rd[sb], (uint32_t)((j / kSBufs - 1) & 1), abort_flag, status, 117))
           break;
         if (!mbar_wait(&sm.kv_full[s], (uint32_t)((j / kStages) & 1), abort_flag, status, 114)) break;
         tc_fence_after();
@@ -400,13 +421,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       const int J = ok ? sm.n_tiles : 0;
       const uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
       for (int j = 0; j < J; ++j) {
-        const int sb = j % kSBufs;
-        if (!mbar_wait(&sm.p_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 115)) break;
+        const int pb = j % kPBufs;
+        if (!mbar_wait(&sm.p_full[pb], (uint32_t)((j / kPBufs) & 1), abort_flag, status, 115)) break;
         tc_fence_after();
         const uint32_t vbase = smem_u32(stage0 + (size_t)(j % kStages) * kStageBytes);
-        const uint32_t pcol = tmem + 128 + kTile * sb;
+        const uint32_t pcol = tmem + 128 + kTile * (kSBufs + pb);
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {  // P_hi, then P_lo
+        for (int part = 0; part < 2; ++part) {  // P_hi (columns 0..15 of the P tile), then P_lo (16..31)
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t bdesc = smem_desc_sw128(vbase + ks * 2048, kBlockBytes, 1024);
@@ -414,7 +435,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           }
         }
         mma_commit(&sm.buf_free[j % kStages]);
-        mma_commit(&sm.s_free[sb]);
+        mma_commit(&sm.p_free[pb]);
         if (j < 60) trace_time(status, 192 + j);
       }
       mma_commit(&sm.drain[2]);
@@ -477,13 +498,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         uint32_t v[32];
         tmem_ld32(tmem + lane_addr + 128 + kTile * sb, v);
         tmem_wait_ld();
-        // The partial scores are read: the softmax warp may overwrite the score tile with P.
+        // The partial scores are read: the score MMAs of tile j + kSBufs may overwrite them.
         tc_fence_before();
-        mbar_arrive(&sm.x_sent[sb][quad]);
-        // The other CTA consumed tile j - kXBufs: its incoming buffer c and this CTA's outgoing
-        // buffer c (read by that copy) are free.
+        mbar_arrive(&sm.s_rd[sb]);
+        // The other CTA consumed tile j - kXBufs (its incoming buffer c and this CTA's outgoing
+        // buffer c, read by that copy, are free), and this CTA's softmax warp read it too.
         if (!__all_sync(0xffffffffu, mbar_wait_cluster(&sm.x_empty[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag,
                                                         status, 126)))
+          break;
+        if (j >= kXBufs &&
+            !__all_sync(0xffffffffu, mbar_wait(&sm.x_own[c][quad], (uint32_t)((j / kXBufs - 1) & 1), abort_flag, status, 130)))
           break;
         uint8_t* xo = xout + c * kXBytes;
 #pragma unroll
@@ -492,6 +516,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
+          mbar_arrive(&sm.x_staged[c][quad]);
           bulk_copy_to_cluster(xin_peer + c * kXBytes, smem_u32(xo) + qoff, kXBytes / 4, xfull_peer + 32 * c);
           if (rt == 0 && j < 60) trace_time(status, 300 + j);
         }
@@ -506,44 +531,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       const float sl = (h < P.H) ? P.sink[h] * 1.4426950408889634f : 0.f;
       float m_used = sl;  // running max in log2 units (starts at the sink)
       float l = 1.f;      // running denominator; the sink contributes exp2(sl - m_used) = 1
-      // s_free[i % kSBufs] completes once per PV(i). A parity wait for PV(i) is unambiguous while
-      // PV(i - kSBufs) has been observed and PV(i + kSBufs) cannot have completed, so PV
-      // completions are observed in order: PV(j - kSBufs) at tile j (it completed before the score
-      // MMAs of tile j were issued, so this never blocks; PV(j) is not issued yet), which makes
-      // PV(j - 1) safe to wait for before a rescale, and PV(J - 1) before the epilogue.
+      // p_free[i % kPBufs] completes once per PV(i). A parity wait for PV(i) is unambiguous while
+      // PV(i - kPBufs) has been observed and PV(i + kPBufs) cannot have completed, so PV
+      // completions are observed in order: PV(j - 2) before P of tile j is stored (its P tile is
+      // then free; PV(j) is not issued yet), PV(j - 1) before a rescale, PV(J - 1) before the
+      // epilogue.
+      static_assert(kPBufs == 2, "P tile j is stored once PV(j - 2) completed");
       int pv_seen = 0;  // PV(0 .. pv_seen-1) observed complete
       auto observe_pv = [&](int upto) -> bool {  // observe PV(pv_seen .. upto-1)
         for (; pv_seen < upto; ++pv_seen)
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_free[pv_seen % kSBufs], (uint32_t)((pv_seen / kSBufs) & 1),
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_free[pv_seen % kPBufs], (uint32_t)((pv_seen / kPBufs) & 1),
                                                  abort_flag, status, 124)))
             return false;
         return true;
       };
       for (; j < J; ++j) {
-        const int c = j % kXBufs, sb = j % kSBufs;
-        const uint32_t sa = tmem + lane_addr + 128 + kTile * sb;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 128)))
+        const int c = j % kXBufs;
+        // This CTA's partial scores of the tile (staged by the sender) and the other CTA's.
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_staged[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag, status, 128)))
           break;
-        if (!observe_pv(j - kSBufs + 1)) break;
-        tc_fence_after();
-        uint32_t v[32];
-        tmem_ld32(sa, v);
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_full[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag, status, 127)))
           break;
         if (rt == 0 && j < 60) trace_time(status, 400 + j);
-        tmem_wait_ld();
         // S = S_0 + S_1 (the same sum in both CTAs), scaled to log2 units; padding -> -inf.
         const uint8_t* xi = xin + c * kXBytes;
+        const uint8_t* xm = xout + c * kXBytes;
         const uint32_t mk = sm.mask[j];
         float x[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const uint4 o = *reinterpret_cast<const uint4*>(xi + xoff(h, i));
+          const uint4 m = *reinterpret_cast<const uint4*>(xm + xoff(h, i));
           const float ov[4] = {__uint_as_float(o.x), __uint_as_float(o.y), __uint_as_float(o.z), __uint_as_float(o.w)};
+          const float mv[4] = {__uint_as_float(m.x), __uint_as_float(m.y), __uint_as_float(m.z), __uint_as_float(m.w)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int cc = 4 * i + e;
-            const float sc = (__uint_as_float(v[cc]) + ov[e]) * P.scale_log2;
+            const float sc = (mv[e] + ov[e]) * P.scale_log2;
             x[cc] = ((mk >> cc) & 1u) ? sc : -CUDART_INF_F;
           }
         }
@@ -558,14 +582,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             for (int e = 0; e < w; ++e) r[e] = fmaxf(r[e], r[e + w]);
           mt = r[0];
         }
-        // mt depends on every value the warp loaded from the buffer (and a warp's loads complete
-        // together), so once it is formed the buffer can be armed for tile j + kXBufs and released
-        // to the other CTA.
+        // mt depends on every value the warp loaded from the buffers (and a warp's loads complete
+        // together), so once it is formed the incoming buffer can be armed for tile j + kXBufs and
+        // released to the other CTA, and the outgoing one to the sender.
         asm volatile("" ::"f"(mt) : "memory");
         __syncwarp();
         if (lane == 0) {
           mbar_arrive_expect_tx(&sm.x_full[c][quad], kXBytes / 4);
           mbar_arrive_remote_relaxed(xempty_peer + 32 * c);
+          mbar_arrive(&sm.x_own[c][quad]);
         }
         if (rt == 0 && j < 60) trace_time(status, 500 + j);
         // Lazy rescale: only when this tile raises the row max by more than 2^8. The TMEM accesses
@@ -595,9 +620,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
             m_used = mt;
           }
         }
-        // P = P_hi + P_lo, both bf16: P_hi in columns [0,16) of the tile, P_lo in [16,32). P_hi is p
-        // truncated to bf16 (the high half of its bits); P_lo = p - P_hi is exact in fp32 and is
-        // rounded to bf16, so P_hi + P_lo is within 2^-16 of p relative.
+        // P = P_hi + P_lo, both bf16, in P tile j % kPBufs: P_hi in columns [0,16), P_lo in
+        // [16,32). P_hi is p truncated to bf16 (the high half of its bits); P_lo = p - P_hi is exact
+        // in fp32 and is rounded to bf16, so P_hi + P_lo is within 2^-16 of p relative.
         uint32_t phi[16], plo[16];
         float ps[16];
 #pragma unroll
@@ -614,15 +639,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int e = 0; e < w; ++e) ps[e] += ps[e + w];
         l += ps[0];
-        // The sender has read this tile's partial scores before P overwrites them.
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_sent[sb][quad], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 129)))
-          break;
+        // P tile j % kPBufs was read by PV(j - kPBufs).
+        if (!observe_pv(j - 1)) break;
         tc_fence_after();
-        tmem_st16(sa, phi);
-        tmem_st16(sa + 16, plo);
+        const uint32_t pa = tmem + lane_addr + 128 + kTile * (kSBufs + j % kPBufs);
+        tmem_st16(pa, phi);
+        tmem_st16(pa + 16, plo);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.p_full[sb]);
+        mbar_arrive(&sm.p_full[j % kPBufs]);
         if (rt == 0 && j < 60) trace_time(status, 128 + j);
       }
       if (j == J && !observe_pv(J)) j = -1;
@@ -637,9 +662,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       fin = __all_sync(0xffffffffu, j == J && J > 0);  // every PV observed complete
       mbar_arrive(&sm.epi);
     }
+    if (!fin && lane == 0) sm.epi_bad = 1;
+    uint8_t* srow = stage0 + (size_t)h * kOutRow;  // every gather and MMA reading the stages completed
     if (fin) {
       tc_fence_after();
-      store_rows(P, sm, tmem + lane_addr + 256, sender ? 128 : 0, (int)half, (long long)qi * P.H + h, h, sm.inv_l[h]);
+      finish_rows(P, sm, tmem + lane_addr + 256, sender ? 128 : 0, 4, (int)half, (long long)qi * P.H + h, h,
+                  sm.inv_l[h], srow);
+    }
+    if (!P.out_is_f32) {
+      // bf16: each head row's 512 bytes leave in one bulk store, once both roles staged their halves.
+      fence_proxy_async_smem();
+      named_bar_sync(1, kRoleThreads + kRoleThreads);
+      if (!sender && h < P.H && !sm.epi_bad) {
+        bulk_store_global(static_cast<uint16_t*>(P.out) + ((long long)qi * P.H + h) * P.d + 256 * half, smem_u32(srow), 512);
+        bulk_commit();
+        bulk_wait_read_all();
+      }
     }
   }
   __syncwarp();

@@ -101,7 +101,7 @@ __global__ void topk_merge_kernel(TopkParams P);
 
 // ------------------------------------------------------------------------------ attention (K4/K5)
 
-constexpr int kAttnThreads = 480;         // warps 0..3 gathers, 4-5 score MMAs, 6 PV MMAs, 7..10 exchange, 11..14 softmax
+constexpr int kAttnThreads = 480;         // warps 0..3 gathers, 4-5 score MMAs, 6 PV MMAs, 7..10 senders, 11..14 softmax
 constexpr int kAttnMaxWindow = 1024;
 constexpr int kAttnMaxTopk = 2048;
 constexpr int kAttnMaxCompressed = 2048;  // HCA: visible entries read per query
