@@ -514,7 +514,7 @@ def main(argv=None):
     bytes_launch = per_q[dom] * wl.B
     achieved = bytes_launch / (r["stage_ms"][dom] * 1e-3) / 1e9
     files = {"indexer": ["indexer.cu", "ptx.cuh", "kernels.cuh"],
-             "attention": ["attn.cu", "ptx.cuh", "kernels.cuh"]}[dom]
+             "attention": ["attn.cu", "ptx.cuh", "kernels.cuh", "rope.cuh"]}[dom]
     total_bytes = sum(per_q.values()) * wl.B
     line = {
         "metric": METRIC,
