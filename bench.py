@@ -354,50 +354,67 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
 
 
 def prefill_ledger(wl):
-    """Algorithmic tensor FLOPs of one CSA prefill pass: attention 4*H*reads*d per query (the
-    pages' analytic count) plus the indexer's 2*H_I*d_I per (query, visible entry)."""
+    """Algorithmic tensor FLOPs of one prefill pass: attention 4*H*reads*d per query (the pages'
+    analytic count) plus, for CSA, the indexer's 2*H_I*d_I per (query, visible entry). HCA reads
+    every visible entry and has no indexer."""
     attn = idx = 0
     for t in range(wl.S):
         vis = min((t + 1) // wl.ratio, wl.max_entries)   # entries visible to query t
-        reads = min(wl.W, t + 1) + min(wl.topk, vis)      # window rows + selected entries
+        sel = min(wl.topk, vis) if wl.has_indexer else vis
+        reads = min(wl.W, t + 1) + sel                    # window rows + selected (or all visible) entries
         attn += 4 * wl.H * reads * wl.d
-        idx += 2 * wl.H_I * wl.d_I * vis
+        if wl.has_indexer:
+            idx += 2 * wl.H_I * wl.d_I * vis
     return attn, idx
 
 
 def run_prefill(wl, steps: int, warmup: int):
-    """One CSA prefill pass over S tokens from an empty cache, through the C ABI: both compressor
-    streams, indexer + top-k, sparse attention. Returns ms per pass and per stage."""
+    """One prefill pass over S tokens from an empty cache, through the C ABI. CSA: both compressor
+    streams (C4A), indexer + top-k, sparse attention. HCA: the C128A stream and attention over every
+    visible entry. Returns ms per pass and per stage."""
     from long_context_decode_c4a_b200 import ops
     dev = "cuda"
     inp = make_inputs(wl, device=dev)
     B, S, d, dI, E = wl.B, wl.S, wl.d, wl.d_I, wl.max_entries
-    main_cfg, idx_cfg = ops.compressor_cfg(4, d), ops.compressor_cfg(4, dI)
-    skv = torch.empty(B, 8, 2 * d, dtype=torch.bfloat16, device=dev)
+    csa = wl.has_indexer
+    rows = (1 + wl.overlap) * wl.ratio
+    main_cfg = ops.compressor_cfg(wl.ratio, d)
+    skv = torch.empty(B, rows, (1 + wl.overlap) * d, dtype=torch.bfloat16, device=dev)
     ssc = torch.empty_like(skv)
-    ikv = torch.empty(B, 8, 2 * dI, dtype=torch.bfloat16, device=dev)
-    isc = torch.empty_like(ikv)
     cache = torch.zeros(B, E, d, dtype=torch.bfloat16, device=dev)
-    icache = torch.zeros(B, E, dI, dtype=torch.bfloat16, device=dev)
     start = torch.zeros(B, dtype=torch.int32, device=dev)
-    topk = torch.empty(B, S, wl.topk, dtype=torch.int32, device=dev)
     out = torch.empty(B, S, wl.H, d, dtype=torch.bfloat16, device=dev)
-    ws_i = ops.workspace(ops._lib.CSA_WS_INDEXER_TOPK, B, S, E, wl.topk, dev)
-    ws_a = ops.workspace(ops._lib.CSA_WS_SPARSE_ATTN, B, S, E, wl.topk, dev)
+    if csa:
+        idx_cfg = ops.compressor_cfg(4, dI)
+        ikv = torch.empty(B, 8, 2 * dI, dtype=torch.bfloat16, device=dev)
+        isc = torch.empty_like(ikv)
+        icache = torch.zeros(B, E, dI, dtype=torch.bfloat16, device=dev)
+        topk = torch.empty(B, S, wl.topk, dtype=torch.int32, device=dev)
+        ws_i = ops.workspace(ops._lib.CSA_WS_INDEXER_TOPK, B, S, E, wl.topk, dev)
+        ws_a = ops.workspace(ops._lib.CSA_WS_SPARSE_ATTN, B, S, E, wl.topk, dev)
+        wss = (ws_i, ws_a)
+    else:
+        ws_a = ops.workspace(ops._lib.CSA_WS_HCA_ATTN, B, S, 1, 1, dev)
+        wss = (ws_a,)
 
     def one(evs=None):
         if evs:
             evs[0].record()
         ops.state_reset(main_cfg, skv, ssc)
-        ops.state_reset(idx_cfg, ikv, isc)
         ops.compress(main_cfg, start, inp["kv"], inp["score"], inp["gamma"], skv, ssc, cache)
-        ops.compress(idx_cfg, start, inp["idx_kv"], inp["idx_score"], inp["idx_gamma"], ikv, isc, icache)
+        if csa:
+            ops.state_reset(idx_cfg, ikv, isc)
+            ops.compress(idx_cfg, start, inp["idx_kv"], inp["idx_score"], inp["idx_gamma"], ikv, isc, icache)
         if evs:
             evs[1].record()
-        ops.indexer_topk(inp["pos"], inp["q_idx"], inp["w"], icache, wl.topk, topk_idx=topk, ws=ws_i)
+        if csa:
+            ops.indexer_topk(inp["pos"], inp["q_idx"], inp["w"], icache, wl.topk, topk_idx=topk, ws=ws_i)
         if evs:
             evs[2].record()
-        ops.sparse_attn(inp["pos"], inp["q"], inp["win_kv"], cache, topk, inp["sink"], wl.W, out=out, ws=ws_a)
+        if csa:
+            ops.sparse_attn(inp["pos"], inp["q"], inp["win_kv"], cache, topk, inp["sink"], wl.W, out=out, ws=ws_a)
+        else:
+            ops.hca_attn(inp["pos"], inp["q"], inp["win_kv"], cache, inp["sink"], wl.W, ratio=wl.ratio, out=out, ws=ws_a)
         if evs:
             evs[3].record()
 
@@ -408,11 +425,14 @@ def run_prefill(wl, steps: int, warmup: int):
     for k in range(steps):
         one(evs[k])
     torch.cuda.synchronize()
-    for w in (ws_i, ws_a):
+    for w in wss:
         if ops.device_status(w) != 0:
             raise RuntimeError("device status after the prefill passes")
     per = lambda i, j: statistics.mean(e[i].elapsed_time(e[j]) for e in evs)
-    return dict(ms=per(0, 3), stage_ms={"compress": per(0, 1), "indexer_topk": per(1, 2), "attention": per(2, 3)})
+    stages = {"compress": per(0, 1), "attention": per(2, 3)}
+    if csa:
+        stages["indexer_topk"] = per(1, 2)
+    return dict(ms=per(0, 3), stage_ms=stages)
 
 
 def extra_workloads(args, peaks):
@@ -431,7 +451,7 @@ def extra_workloads(args, peaks):
                                   "unit": "GB/s", "frac": total / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                   "scope": "whole step, algorithmic bytes"}}
         torch.cuda.empty_cache()
-    for name, steps in (("csa_prefill_8k", 3), ("tiny_csa_prefill", 20)):
+    for name, steps in (("csa_prefill_8k", 3), ("hca_prefill_8k", 3), ("tiny_csa_prefill", 20)):
         wl = WORKLOADS[name]
         r = run_prefill(wl, steps, 3)
         attn_f, idx_f = prefill_ledger(wl)
@@ -440,7 +460,7 @@ def extra_workloads(args, peaks):
                      "kernels_ms": r["stage_ms"],
                      "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                   "frac": tf / peaks["bf16_tflops"], "flops_per_pass": attn_f + idx_f,
-                                  "scope": "whole pass, algorithmic FLOPs (attention 4*H*reads*d + indexer)"}}
+                                  "scope": "whole pass, algorithmic FLOPs (attention 4*H*reads*d + CSA indexer)"}}
         torch.cuda.empty_cache()
     return res
 

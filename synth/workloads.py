@@ -87,6 +87,9 @@ WORKLOADS: Dict[str, Workload] = {
     "csa_prefill_8k": Workload("csa_prefill_8k", "csa_prefill", B=1, S=8192, ctx=8192),
     # B=8 requests at position 1048575: 262144 entries per request.
     "long_csa_decode_1m": Workload("long_csa_decode_1m", "csa_decode", B=8, S=1, ctx=1048576),
+    # B=1, S=8192 new tokens from an empty cache through the HCA layer: ratio 128 without overlap
+    # (64 entries), every visible entry read, no indexer.
+    "hca_prefill_8k": Workload("hca_prefill_8k", "hca_prefill", B=1, S=8192, ctx=8192, ratio=128, H_I=0, topk=0),
 }
 
 

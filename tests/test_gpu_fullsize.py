@@ -115,6 +115,25 @@ def test_csa_prefill_8k_sampled(ops):
         assert_attn_close(res["out"][0, i], ref_out, f"prefill query {i}")
 
 
+def test_hca_prefill_8k_sampled(ops):
+    """S = 8192 tokens through the HCA layer from an empty cache: all 64 entries, sampled queries."""
+    from tests.test_gpu_layer import run_hca_prefill
+    wl = WORKLOADS["hca_prefill_8k"]
+    inp = make_inputs(wl, device="cuda")
+    res = run_hca_prefill(ops, wl, inp)
+    cfg = O.CompressorCfg(wl.ratio, wl.d)
+    ent = O.compress_parallel(cfg, np64(inp["kv"][0]), np64(inp["score"][0]), np64(inp["gamma"]))
+    assert_compress_close(res["cache32"][0], res["cache"][0], ent, "hca prefill entries")
+    cache = O.bf16(ent)
+    ring = RowSource(inp["win_kv"][0])
+    sink = np64(inp["sink"])
+    for i in (0, 127, 128, 4095, 4096, 6000, 8190, 8191):
+        t = i
+        ref_out = O.attend_query(np64(inp["q"][0, i]), t, wl.W, ring, wl.S, cache, list(range((t + 1) // wl.ratio)),
+                                 sink, 1 / math.sqrt(wl.d), 64, 10000.0)
+        assert_attn_close(res["out"][0, i], ref_out, f"hca prefill query {i}")
+
+
 def test_long_context_decode_sampled(ops):
     """B = 8 requests at position 1,048,575 (262,144 entries each): the chunked top-k path."""
     wl = WORKLOADS["long_csa_decode_1m"]

@@ -184,3 +184,40 @@ def test_prefill_medium_end_to_end(ops):
     inp = make_inputs(wl)
     res = run_csa_prefill(ops, wl, {k: v.cuda() for k, v in inp.items()})
     check_prefill_queries(wl, O.to_numpy_inputs(inp), res, [0, 2, 3, 4, 63, 127, 128, 255, 256, 511, 998, 999])
+
+
+def run_hca_prefill(ops, wl, inp):
+    """HCA prefill through the C ABI: the C128A stream over the segment, then attention over the
+    window and every visible entry."""
+    B, S, d = wl.B, wl.S, wl.d
+    dev = "cuda"
+    E = wl.max_entries
+    cfg = ops.compressor_cfg(wl.ratio, d)
+    skv = torch.empty(B, wl.ratio, d, dtype=torch.bfloat16, device=dev)
+    ssc = torch.empty_like(skv)
+    ops.state_reset(cfg, skv, ssc)
+    cache = torch.zeros(B, E, d, dtype=torch.bfloat16, device=dev)
+    cache32 = torch.zeros(B, E, d, dtype=torch.float32, device=dev)
+    start = torch.zeros(B, dtype=torch.int32, device=dev)
+    ops.compress(cfg, start, inp["kv"], inp["score"], inp["gamma"], skv, ssc, cache, cache32)
+    out = torch.empty(B, S, wl.H, d, dtype=torch.float32, device=dev)
+    ops.hca_attn(inp["pos"], inp["q"], inp["win_kv"], cache, inp["sink"], wl.W, ratio=wl.ratio, out=out)
+    torch.cuda.synchronize()
+    return dict(cache=cache, cache32=cache32, out=out, state_kv=skv)
+
+
+def check_hca_prefill_queries(wl, inp_np, res, queries):
+    ref = O.csa_prefill(inp_np, 0, queries, H=wl.H, d=wl.d, W=wl.W, topk=0, ratio=wl.ratio, with_indexer=False)
+    assert_compress_close(res["cache32"][0], res["cache"][0], ref["entries"], "hca prefill entries")
+    for i in queries:
+        assert_attn_close(res["out"][0, i], ref["queries"][i]["out"], f"hca prefill query {i}")
+
+
+def test_hca_prefill_medium_end_to_end(ops):
+    """S = 1000 tokens through the HCA layer (ratio 128: 7 entries, a ragged last group), queries at
+    every point where an entry becomes visible and at the window edges."""
+    wl = WORKLOADS["hca_prefill_8k"].scaled(S=1000, ctx=1000)
+    inp = make_inputs(wl)
+    res = run_hca_prefill(ops, wl, {k: v.cuda() for k, v in inp.items()})
+    queries = [0, 1, 126, 127, 128, 129, 255, 256, 383, 384, 511, 639, 640, 767, 895, 896, 998, 999]
+    check_hca_prefill_queries(wl, O.to_numpy_inputs(inp), res, queries)

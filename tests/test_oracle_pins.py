@@ -299,6 +299,24 @@ def test_topk_at_least_visible_reduces_to_dense_attention():
         assert np.allclose(res["queries"][i]["out"], ref, atol=1e-10)
 
 
+def test_hca_prefill_is_dense_attention_over_every_visible_entry():
+    """HCA ([P5] §3, no index module): the prefill path without the indexer (C128A, ratio 128, no
+    overlap) equals dense attention over the window and every visible entry, written out
+    independently of the oracle's candidate gathering."""
+    rng = np.random.default_rng(11)
+    S, H, d, W, ratio = 300, 4, 512, 16, 128
+    inp = dict(kv=rng.standard_normal((1, S, d)), score=rng.standard_normal((1, S, d)),
+               win_kv=rng.standard_normal((1, S, d)), q=rng.standard_normal((1, S, H, d)) / math.sqrt(d) * 3,
+               sink=rng.standard_normal(H), gamma=np.ones(d), pos=np.arange(S)[None, :])
+    qs = [0, 126, 127, 128, 255, 256, 299]
+    res = O.csa_prefill(inp, 0, qs, H=H, d=d, W=W, topk=0, ratio=ratio, with_indexer=False)
+    assert res["cache"].shape == (S // ratio, d)
+    for i in qs:
+        ref = _dense_reference(inp["q"][0, i], i, W, inp["win_kv"][0], S, res["cache"], (i + 1) // ratio,
+                               inp["sink"], 1 / math.sqrt(d), 64, 10000.0)
+        assert np.allclose(res["queries"][i]["out"], ref, atol=1e-10)
+
+
 def test_future_group_values_do_not_leak():
     """T4: adversarial values in an incomplete group (and later tokens) do not change the
     output of any query that precedes the group's completion."""
