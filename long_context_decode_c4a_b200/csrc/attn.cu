@@ -18,21 +18,23 @@
 // S_0 + S_1 (the same sum in both, fp addition being commutative), run the same online softmax,
 // and accumulate O[:, half] += P V[:, half].
 //   TMEM (512 columns): [0,128) Q[:, half] as bf16 pairs (A operand of the score TS-MMAs);
-//     [128,256) four 32-column score tiles (partial scores, then P_hi in columns [0,16) and P_lo
-//     in [16,32)); [256,512) O[:, half].
+//     [128,192) two 32-column partial-score tiles, rewritten once the senders have loaded them;
+//     [192,256) two 32-column P tiles (P_hi in columns [0,16), P_lo in [16,32)), the A operand of
+//     the PV TS-MMAs; [256,512) O[:, half].
 //   SMEM: eight 16 KB stages of 32 half-rows (4 blocks of 64 dims in the 128B-swizzled layout that
 //     serves S as a K-major B operand and PV as an MN-major B operand); two 16 KB outgoing and two
 //     16 KB incoming exchange buffers (together they first stage Q[:, half] on its way into TMEM);
-//     the candidate list.
+//     the candidate list. At the end the stages stage the bf16 output rows.
 //   Warps: 0..3 build the candidate list and gather half-rows with coalesced 16-byte cp.async,
 //     announcing each tile as soon as it lands; 4 and 5 issue the score MMAs of even and odd tiles
 //     (one thread issues a tcgen05.mma only every ~50 cycles); 6 issues the PV MMAs in tile order
-//     (and owns TMEM); 7..10 send the partial scores of their 32 heads (one 4 KB bulk copy per warp
-//     and tile, into the same quadrant's rows of the other CTA's incoming buffer); 11..14 add the
-//     incoming partial scores to their own and run the softmax. A sender and a softmax warp of the
-//     same TMEM lane quadrant trade with the two warps of that quadrant in the other CTA, with
-//     barriers of their own, so the four quadrants run independently; sending tile j+1 overlaps
-//     receiving tile j. Warps 7..14 own one head (TMEM lane) per thread and share the epilogue.
+//     (and owns TMEM); 7..10 load the partial scores of their 32 heads, free the score tile, stage
+//     the 4 KB in the outgoing buffer and bulk-copy it into the same quadrant's rows of the other
+//     CTA's incoming buffer; 11..14 add this CTA's staged partial scores and the other CTA's, run
+//     the softmax and store P. A sender and a softmax warp of the same TMEM lane quadrant trade
+//     with the two warps of that quadrant in the other CTA, with barriers of their own, so the four
+//     quadrants run independently. Warps 7..14 own one head (TMEM lane) per thread and share the
+//     epilogue.
 // Precision: P = P_hi + P_lo with both parts in bf16 (about 16 significant bits), accumulated by two
 // PV MMAs; a single bf16 P (8 bits) leaves errors near 1% of the output RMS on short candidate sets.
 // Online softmax in the log2 domain; the running max starts at the sink; O is rescaled only when a
