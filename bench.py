@@ -435,6 +435,36 @@ def run_prefill(wl, steps: int, warmup: int):
     return dict(ms=per(0, 3), stage_ms=stages)
 
 
+def run_output_projection(M: int, steps: int, warmup: int):
+    """The grouped output projection on M rows of the Pro shapes through the C ABI (two GEMM launches,
+    plus a zeroing launch when the second contraction is split over K). Returns ms per call."""
+    from long_context_decode_c4a_b200 import ops
+    from synth.workloads import make_oproj_inputs
+    inp = make_oproj_inputs(M, device="cuda")
+    G, R, Kg = inp["wo_a"].shape
+    D = inp["wo_b"].shape[0]
+    r = torch.empty(M, G * R, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(M, D, dtype=torch.float32, device="cuda")
+    ws = ops.workspace(ops._lib.CSA_WS_OUTPUT_PROJ, 1, 1, 1, 1, "cuda")
+    for _ in range(warmup):
+        ops.output_projection(inp["o"], inp["wo_a"], inp["wo_b"], r, y, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        ops.output_projection(inp["o"], inp["wo_a"], inp["wo_b"], r, y, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    if ops.device_status(ws) != 0:
+        raise RuntimeError("device status after the output projection")
+    ms = e0.elapsed_time(e1) / steps
+    weights = (G * R * Kg + D * G * R) * 2
+    traffic = weights + M * G * Kg * 2 + 2 * M * G * R * 2 + M * D * 4
+    flops = 2 * M * (G * R * Kg + D * G * R)
+    del inp, r, y
+    return ms, traffic, flops
+
+
 def extra_workloads(args, peaks):
     """Short measurements of the other synthetic configurations (one GPU, same process)."""
     res = {}
@@ -461,6 +491,23 @@ def extra_workloads(args, peaks):
                      "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                   "frac": tf / peaks["bf16_tflops"], "flops_per_pass": attn_f + idx_f,
                                   "scope": "whole pass, algorithmic FLOPs (attention 4*H*reads*d + CSA indexer)"}}
+        torch.cuda.empty_cache()
+    # The grouped output projection after the path ([P1] "输出投影也分组"): decode rows stream the
+    # 176 Mi weights (HBM-bound); prefill rows are a dense contraction (tensor-bound).
+    for name, M, steps in (("output_projection_decode_b64", 64, 20), ("output_projection_prefill_8k", 8192, 3)):
+        ms, traffic, flops = run_output_projection(M, steps, 3)
+        if M <= 256:
+            ach = traffic / (ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "bytes_per_call": traffic,
+                    "scope": "weights + o + r (written and read) + y, algorithmic bytes"}
+        else:
+            ach = flops / (ms * 1e-3) / 1e12
+            roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": ach / peaks["bf16_tflops"], "flops_per_call": flops,
+                    "scope": "2*M*(G*R*Kg + D*G*R)"}
+        res[name] = {"value": M * 1000.0 / ms, "unit": "rows/s", "ms_per_step": ms, "rows": M,
+                     "shape": "G=16 groups x Kg=4096 -> R=1024, then 16384 -> D=7168", "roofline": roof}
         torch.cuda.empty_cache()
     return res
 

@@ -83,7 +83,8 @@ enum {
   CSA_WS_SPARSE_ATTN = 2,
   CSA_WS_HCA_ATTN = 3,
   CSA_WS_DECODE_FUSED = 4,
-  CSA_WS_HCA_DECODE_FUSED = 5
+  CSA_WS_HCA_DECODE_FUSED = 5,
+  CSA_WS_OUTPUT_PROJ = 6
 };
 
 /*
@@ -295,6 +296,25 @@ CSA_API int hca_decode_fused(const hca_decode_args* a, void* stream);
 CSA_API int csa_indexer_topk_noalloc(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
                                      const uint16_t* q_idx, const float* w, const uint16_t* idx_cache,
                                      int64_t idx_bstride, int max_entries, int32_t* topk_idx, void* stream);
+
+/*
+ * csa_output_projection -- the grouped output projection after the inverse RoPE ([P1] section
+ * "输出投影也分组，并且降低中间维度"): the M = B*S output rows o [M, G*Kg] (G groups of 8 heads, Kg = 8*d)
+ * are projected per group, r[m, g*R + i] = sum_k o[m, g*Kg + k] * wo_a[g*R + i, k], then
+ * y[m, j] = sum_c r[m, c] * wo_b[j, c]. Pro: G = 16, Kg = 4096, R = 1024, D = 7168.
+ *   o      dev bf16 [M, G*Kg] (the attention output [B, S, H, d] read as rows of H*d).
+ *   wo_a   dev bf16 [G*R, Kg] (Wo_a [G, R, Kg]).   wo_b: dev bf16 [D, G*R].
+ *   r      dev bf16 [M, G*R], written (r is rounded to bf16 before the second product).
+ *   y      dev float [M, D], written.
+ *   ws/ws_bytes: workspace of at least csa_workspace_size(CSA_WS_OUTPUT_PROJ, ...) (status word).
+ * Supported: Kg and G*R multiples of 64, R and D multiples of 128, M <= 8,388,480 (65535 tiles of
+ * 128 rows). Alignment: every pointer 16 bytes. Contractions run on the tensor cores with fp32
+ * accumulation; the order of the fp32 additions differs from a sequential sum.
+ * Returns CSA_ERR_INVALID_ARG / CSA_ERR_UNSUPPORTED without launching on bad arguments.
+ */
+CSA_API int csa_output_projection(int M, int G, int Kg, int R, int D, const uint16_t* o, const uint16_t* wo_a,
+                                  const uint16_t* wo_b, uint16_t* r, float* y, void* ws, size_t ws_bytes,
+                                  void* stream);
 
 /*
  * csa_get_device_status -- synchronise `stream`, read the status word in `ws` into *status

@@ -26,6 +26,7 @@ CSA_WS_SPARSE_ATTN = 2
 CSA_WS_HCA_ATTN = 3
 CSA_WS_DECODE_FUSED = 4
 CSA_WS_HCA_DECODE_FUSED = 5
+CSA_WS_OUTPUT_PROJ = 6
 
 
 class CompressorCfg(ctypes.Structure):
@@ -86,6 +87,8 @@ PROTOTYPES = {
     "csa_get_device_status": (c_int, [c_void_p, c_void_p, POINTER(c_int)]),
     "csa_indexer_topk_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                                          c_void_p, c_int64, c_int, c_void_p, c_void_p]),
+    "csa_output_projection": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_void_p, c_size_t, c_void_p]),
 }
 
 _lib = None

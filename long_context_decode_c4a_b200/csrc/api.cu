@@ -127,6 +127,7 @@ int device_info(DeviceInfo** out) {
       return fail(CSA_ERR_UNSUPPORTED, "libcsa is built for sm_100a; device is sm_%d%d", cc_major, cc_minor);
     const int ms = d.max_smem;
     CSA_CUDA(cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
+    CSA_CUDA(cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
     CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
     CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
     CSA_CUDA(cudaFuncSetAttribute(indexer_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, ms));
@@ -439,6 +440,25 @@ int run_attn(const AttnArgs& a, bool csa_mode, cudaStream_t st) {
   return CSA_OK;
 }
 
+// C = A . B^T on the tensor cores (gemm_kernel). A [a_rows, a_cols] and B [b_rows, b_cols] are
+// row-major bf16 with pitches lda / ldb; `groups` independent products along blockIdx.z.
+int run_gemm(const void* A, uint64_t a_cols, uint64_t a_rows, uint64_t lda, const void* Bm, uint64_t b_cols,
+             uint64_t b_rows, uint64_t ldb, GemmParams P, int groups, int sms, cudaStream_t st) {
+  CUtensorMap map_a, map_b;
+  if (int rc = make_map_2d(&map_a, A, a_cols, a_rows, lda, 64, 128)) return rc;
+  if (int rc = make_map_2d(&map_b, Bm, b_cols, b_rows, ldb, 64, 128)) return rc;
+  const unsigned mt = (unsigned)((P.M + 127) / 128);
+  CSA_CHECK_SUP(mt <= 65535u, "too many rows");
+  const dim3 grid((unsigned)(P.N / 128), mt, (unsigned)(groups * P.splits));
+  if (P.c_mode == kGemmOutF32Add) {
+    const long long n4 = (long long)P.M * P.ldc / 4;
+    const int blocks = (int)std::min<long long>((n4 + 255) / 256, 4LL * sms);
+    CSA_CUDA(launch_pdl(zero_f32_kernel, dim3(blocks), dim3(256), 0, st, static_cast<float*>(P.c), n4));
+  }
+  CSA_CUDA(launch_pdl(gemm_kernel, grid, dim3(kGemmThreads), gemm_smem_bytes(), st, map_a, map_b, P));
+  return CSA_OK;
+}
+
 }  // namespace
 }  // namespace csa
 
@@ -475,6 +495,7 @@ int csa_workspace_size(int kind, int B, int S, int max_entries, int topk, size_t
     case CSA_WS_SPARSE_ATTN:
     case CSA_WS_HCA_ATTN:
     case CSA_WS_HCA_DECODE_FUSED:
+    case CSA_WS_OUTPUT_PROJ:
       *bytes = kStatusBytes;
       return CSA_OK;
     default:
@@ -533,6 +554,55 @@ int hca_attn(int B, int S, int H, int d, int rope_dim, float rope_base, float sc
              cache_bstride, max_entries, nullptr, 0, sink, out, out_is_f32, ws, ws_bytes};
   if (int rc = check_attn_args(a, false)) return rc;
   return run_attn(a, false, static_cast<cudaStream_t>(stream));
+}
+
+int csa_output_projection(int M, int G, int Kg, int R, int D, const uint16_t* o, const uint16_t* wo_a,
+                          const uint16_t* wo_b, uint16_t* r, float* y, void* ws, size_t ws_bytes, void* stream) {
+  CSA_CHECK_ARG(M > 0 && G > 0 && Kg > 0 && R > 0 && D > 0, "sizes must be positive");
+  CSA_CHECK_ARG(o && wo_a && wo_b && r && y, "null pointer");
+  CSA_CHECK_ARG(aligned(o, 16) && aligned(wo_a, 16) && aligned(wo_b, 16) && aligned(r, 16) && aligned(y, 16),
+                "pointers must be 16-byte aligned");
+  CSA_CHECK_SUP(Kg % 64 == 0 && (G * R) % 64 == 0, "Kg and G*R must be multiples of 64");
+  CSA_CHECK_SUP(R % 128 == 0 && D % 128 == 0, "R and D must be multiples of 128");
+  CSA_CHECK_SUP((long long)G * Kg <= (1LL << 31) && (long long)G * R <= (1LL << 31), "too wide");
+  if (int rc = check_ws(ws, ws_bytes, kStatusBytes)) return rc;
+  DeviceInfo* dev;
+  if (int rc = device_info(&dev)) return rc;
+  CSA_CHECK_SUP(gemm_smem_bytes() <= (size_t)dev->max_smem, "shared memory too small for the GEMM kernel");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  // r = o . Wo_a^T per group (bf16 out).
+  GemmParams P1{};
+  P1.M = M;
+  P1.N = R;
+  P1.K = Kg;
+  P1.splits = 1;
+  P1.a_group_cols = Kg;
+  P1.b_group_rows = R;
+  P1.c_group_cols = R;
+  P1.ldc = (long long)G * R;
+  P1.c = r;
+  P1.c_mode = kGemmOutBf16;
+  P1.status = status;
+  if (int rc = run_gemm(o, (uint64_t)G * Kg, (uint64_t)M, (uint64_t)G * Kg, wo_a, (uint64_t)Kg, (uint64_t)G * R,
+                        (uint64_t)Kg, P1, G, dev->sms, st))
+    return rc;
+  // y = r . Wo_b^T; when the output tiles alone would leave SMs idle, K is split (fp32 reduction).
+  const long long tiles = (long long)(D / 128) * ((M + 127) / 128);
+  const int kblocks = G * R / 64;
+  int splits = 1;
+  while (splits < 8 && tiles * splits * 2 <= dev->sms && kblocks % (splits * 2) == 0) splits *= 2;
+  GemmParams P2{};
+  P2.M = M;
+  P2.N = D;
+  P2.K = G * R;
+  P2.splits = splits;
+  P2.ldc = D;
+  P2.c = y;
+  P2.c_mode = splits > 1 ? kGemmOutF32Add : kGemmOutF32;
+  P2.status = status;
+  return run_gemm(r, (uint64_t)G * R, (uint64_t)M, (uint64_t)G * R, wo_b, (uint64_t)G * R, (uint64_t)D,
+                  (uint64_t)G * R, P2, 1, dev->sms, st);
 }
 
 int csa_decode_fused(const csa_decode_args* a, void* stream) {

@@ -129,7 +129,32 @@ struct AttnParams {
 
 __global__ void attn_kernel(const __grid_constant__ CUtensorMap map_q, AttnParams P);
 
+// ------------------------------------------------------------------------------ output projection
+
+constexpr int kGemmThreads = 128;
+constexpr int kGemmStages = 6;
+constexpr int kGemmOutBf16 = 0;           // C stored as bf16
+constexpr int kGemmOutF32 = 1;            // C stored as fp32
+constexpr int kGemmOutF32Add = 2;         // C += tile (fp32 reduction; C zeroed first), for split K
+
+// C[m, g*c_group_cols + n] = sum_k A[m, g*a_group_cols + k] * B[g*b_group_rows + n, k] over this CTA's
+// K split; A, B through the tensor maps (bf16, 128B swizzle, boxes of 64 x 128).
+struct GemmParams {
+  int M, N, K;                            // rows of C, columns of C per group, K per group
+  int splits;                             // K splits (blockIdx.z = group * splits + split)
+  int a_group_cols, b_group_rows, c_group_cols;
+  long long ldc;                          // row pitch of C (elements)
+  void* c;
+  int c_mode;
+  uint32_t* status;
+};
+
+__global__ void gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                            GemmParams P);
+__global__ void zero_f32_kernel(float* p, long long n4);
+
 size_t attn_smem_bytes();
+size_t gemm_smem_bytes();
 size_t indexer_smem_bytes(int stages, int N);
 
 }  // namespace csa

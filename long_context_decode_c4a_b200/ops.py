@@ -356,6 +356,32 @@ def hca_decode_fused(st: "HcaDecodeState", pos, kv, score, win_kv, q, sink, out=
     return out
 
 
+def output_projection(o: torch.Tensor, wo_a: torch.Tensor, wo_b: torch.Tensor, r: Optional[torch.Tensor] = None,
+                      y: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """Grouped output projection: o holds M rows of G*Kg bf16 values ([B, S, H, d] or [M, G*Kg]),
+    wo_a [G, R, Kg] and wo_b [D, G*R] bf16. Returns (r [M, G*R] bf16, y [M, D] fp32)."""
+    G, R, Kg = wo_a.shape
+    D = wo_b.shape[0]
+    _need(wo_a, "wo_a", torch.bfloat16)
+    _need(wo_b, "wo_b", torch.bfloat16, (D, G * R))
+    _need(o, "o", torch.bfloat16)
+    if o.numel() % (G * Kg) != 0:
+        raise ValueError("o must hold whole rows of G*Kg values")
+    M = o.numel() // (G * Kg)
+    if r is None:
+        r = torch.empty(M, G * R, dtype=torch.bfloat16, device=o.device)
+    if y is None:
+        y = torch.empty(M, D, dtype=torch.float32, device=o.device)
+    _need(r, "r", torch.bfloat16, (M, G * R))
+    _need(y, "y", torch.float32, (M, D))
+    if ws is None:
+        ws = workspace(_lib.CSA_WS_OUTPUT_PROJ, 1, 1, 1, 1, o.device)
+    check(_lib.load().csa_output_projection(M, G, Kg, R, D, o.data_ptr(), wo_a.data_ptr(), wo_b.data_ptr(),
+                                            r.data_ptr(), y.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
+          "csa_output_projection")
+    return r, y
+
+
 def device_status(ws: torch.Tensor) -> int:
     """Synchronise the current stream, read and clear the workspace's device status word."""
     st = ctypes.c_int(0)

@@ -183,3 +183,20 @@ def make_inputs(wl: Workload, device: str = "cpu", seed: Optional[int] = None) -
     if wl.has_indexer:
         out["idx_gamma"] = torch.ones(dI, dtype=torch.bfloat16, device=device)
     return out
+
+
+# Grouped output projection ([P1] "输出投影也分组"): Pro shapes.
+OPROJ_GROUPS, OPROJ_KG, OPROJ_R, OPROJ_D = 16, 4096, 1024, 7168
+
+
+def make_oproj_inputs(M: int, G: int = OPROJ_GROUPS, Kg: int = OPROJ_KG, R: int = OPROJ_R, D: int = OPROJ_D,
+                      seed: int = 0, device: str = "cpu") -> Dict[str, torch.Tensor]:
+    """Seeded inputs of the output projection: o [M, G*Kg] ~ bf16 N(0,1) / 4 (the attention output is a
+    convex combination of cache rows, smaller than a row), random weights Wo_a [G, R, Kg] ~ N(0,1)/sqrt(Kg)
+    and Wo_b [D, G*R] ~ N(0,1)/sqrt(G*R), bf16. Draw order: o, Wo_a, Wo_b."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    o = _randn(gen, (M, G * Kg), device, dtype=torch.float32).mul_(0.25).to(torch.bfloat16)
+    wa = _randn(gen, (G, R, Kg), device, dtype=torch.float32).mul_(1.0 / math.sqrt(Kg)).to(torch.bfloat16)
+    wb = _randn(gen, (D, G * R), device, dtype=torch.float32).mul_(1.0 / math.sqrt(G * R)).to(torch.bfloat16)
+    return {"o": o, "wo_a": wa, "wo_b": wb}

@@ -28,7 +28,8 @@ def declared_symbols():
 def test_header_declares_the_boundary():
     names = declared_symbols()
     for want in ("csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode_fused",
-                 "hca_decode_fused", "csa_workspace_size", "csa_get_device_status", "csa_state_reset"):
+                 "hca_decode_fused", "csa_workspace_size", "csa_get_device_status", "csa_state_reset",
+                 "csa_output_projection"):
         assert want in names
 
 
@@ -82,6 +83,8 @@ def test_workspace_sizes(lib):
     assert n.value >= 256 + 8 * 262144 * 4 + 2 * 8 * 16 * 1024 * 4
     assert lib.csa_workspace_size(_lib.CSA_WS_HCA_ATTN, 64, 1, 256, 0, ctypes.byref(n)) == 0
     assert n.value == 256
+    assert lib.csa_workspace_size(_lib.CSA_WS_OUTPUT_PROJ, 1, 1, 1, 1, ctypes.byref(n)) == 0
+    assert n.value == 256
     assert lib.csa_workspace_size(99, 1, 1, 1, 1, ctypes.byref(n)) == _lib.CSA_ERR_INVALID_ARG
     assert lib.csa_workspace_size(_lib.CSA_WS_DECODE_FUSED, 0, 1, 1, 1, ctypes.byref(n)) == _lib.CSA_ERR_INVALID_ARG
 
@@ -125,4 +128,15 @@ def test_host_side_argument_checks_launch_nothing(lib):
     assert lib.csa_decode_fused(ctypes.byref(a), null) in (_lib.CSA_ERR_INVALID_ARG, _lib.CSA_ERR_UNSUPPORTED)
     st = ctypes.c_int()
     assert lib.csa_get_device_status(None, null, ctypes.byref(st)) == _lib.CSA_ERR_INVALID_ARG
+    # output projection: null pointers, misalignment, unsupported widths, missing workspace
+    assert lib.csa_output_projection(64, 16, 4096, 1024, 7168, null, 16, 16, 16, 16, 256, 256, null) == \
+        _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_output_projection(64, 16, 4096, 1024, 7168, 24, 16, 16, 16, 16, 256, 256, null) == \
+        _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_output_projection(64, 16, 4000, 1024, 7168, 16, 16, 16, 16, 16, 256, 256, null) == \
+        _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_output_projection(64, 16, 4096, 1000, 7168, 16, 16, 16, 16, 16, 256, 256, null) == \
+        _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_output_projection(64, 16, 4096, 1024, 7168, 16, 16, 16, 16, 16, null, 0, null) == \
+        _lib.CSA_ERR_WORKSPACE
     assert lib.csa_last_error()

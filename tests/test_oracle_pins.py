@@ -378,3 +378,51 @@ def test_rmsnorm_eps_matters_for_small_vectors():
     y = O.rms_norm(x, 1.0, 1e-6)
     assert np.allclose(y, 1e-4 / math.sqrt(1e-8 + 1e-6), rtol=1e-12)
     assert np.array_equal(O.rms_norm(np.zeros(8), 1.0, 1e-6), np.zeros(8))
+
+
+# ----------------------------------------------------------------------------- output projection
+
+def test_output_projection_one_hot_weights_select_values():
+    """[P1] "输出投影也分组": with Wo_a[g] selecting dims perm_g of its group and Wo_b a permutation,
+    y picks single entries of o, so every index of the grouped einsum and the flatten is checked."""
+    rng = np.random.default_rng(20)
+    M, G, Kg, R = 3, 4, 16, 8
+    D = G * R
+    o = O.bf16(rng.standard_normal((M, G * Kg)))
+    wa = np.zeros((G, R, Kg))
+    sel = [rng.choice(Kg, R, replace=False) for _ in range(G)]
+    for g in range(G):
+        wa[g, np.arange(R), sel[g]] = 1.0
+    perm = rng.permutation(G * R)
+    wb = np.zeros((D, G * R))
+    wb[np.arange(D), perm] = 1.0
+    r, rb, y = O.output_projection(o, wa, wb)
+    for m in range(M):
+        for g in range(G):
+            for i in range(R):
+                assert r[m, g * R + i] == o[m, g * Kg + sel[g][i]]
+        for j in range(D):
+            c = perm[j]
+            assert y[m, j] == o[m, (c // R) * Kg + sel[c // R][c % R]]
+
+
+def test_output_projection_groups_are_independent_and_linear():
+    """Changing the input of one group changes only that group's block of r; the bf16 rounding of
+    r (R15) commutes with a power-of-two scale, so y scales exactly."""
+    rng = np.random.default_rng(21)
+    M, G, Kg, R, D = 2, 3, 32, 8, 5
+    o = O.bf16(rng.standard_normal((M, G * Kg)))
+    wa = O.bf16(rng.standard_normal((G, R, Kg)))
+    wb = O.bf16(rng.standard_normal((D, G * R)))
+    r, rb, y = O.output_projection(o, wa, wb)
+    o2 = o.copy()
+    o2[:, Kg:2 * Kg] += 1.0
+    r2, _, _ = O.output_projection(o2, wa, wb)
+    changed = np.any(r2 != r, axis=0)
+    assert not changed[:R].any() and changed[R:2 * R].any() and not changed[2 * R:].any()
+    _, rb4, y4 = O.output_projection(4.0 * o, wa, wb)
+    assert np.array_equal(rb4, 4.0 * rb) and np.allclose(y4, 4.0 * y, rtol=0, atol=1e-12 * np.abs(y).max())
+    # r is exactly the per-group matrix product before rounding; y uses the rounded r
+    for g in range(G):
+        assert np.allclose(r[:, g * R:(g + 1) * R], o[:, g * Kg:(g + 1) * Kg] @ wa[g].T, rtol=1e-14, atol=1e-12)
+    assert np.array_equal(rb, O.bf16(r))
