@@ -33,7 +33,7 @@ Where the pages are silent the oracle takes one reading, named READING-n below:
       entries, every visible entry is taken.
   R13 ties in the indexer score go to the lower index; -0 equals +0; NaN sorts lowest.
   R14 the compressor scores are used as given (no extra bias).
-  R15 output projection: the intermediate r of each group is rounded to bf16 before the second
+  R20 output projection: the intermediate r of each group is rounded to bf16 before the second
       product (the pages give the two einsums, not the precision between them).
 """
 
@@ -309,7 +309,7 @@ def attend_query(q_t: np.ndarray, t: int, W: int, ring, ring_cap, cache, selecte
 def output_projection(o_rows: np.ndarray, wo_a: np.ndarray, wo_b: np.ndarray):
     """[P1] "输出投影也分组，并且降低中间维度": the rows o [M, G*Kg] (the inverse-RoPE'd output of
     groups of 8 heads) are reshaped to [M, G, Kg]; r[m, g, i] = sum_k o[m, g, k] * Wo_a[g, i, k]
-    (einsum "bsgd,grd->bsgr"); y = r.flatten(1) @ Wo_b^T. r is rounded to bf16 first (R15).
+    (einsum "bsgd,grd->bsgr"); y = r.flatten(1) @ Wo_b^T. r is rounded to bf16 first (R20).
     Returns (r in float64, r rounded to bf16, y)."""
     M = o_rows.shape[0]
     G, R, Kg = wo_a.shape

@@ -408,7 +408,7 @@ def test_output_projection_one_hot_weights_select_values():
 
 def test_output_projection_groups_are_independent_and_linear():
     """Changing the input of one group changes only that group's block of r; the bf16 rounding of
-    r (R15) commutes with a power-of-two scale, so y scales exactly."""
+    r (R20) commutes with a power-of-two scale, so y scales exactly."""
     rng = np.random.default_rng(21)
     M, G, Kg, R, D = 2, 3, 32, 8, 5
     o = O.bf16(rng.standard_normal((M, G * Kg)))
