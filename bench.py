@@ -465,6 +465,35 @@ def run_output_projection(M: int, steps: int, warmup: int):
     return ms, traffic, flops
 
 
+def run_q_path(M: int, steps: int, warmup: int):
+    """The low-rank query path on M tokens of the Pro shapes through the C ABI (two GEMMs, the row
+    RMSNorm and the per-head norm with RoPE). Returns ms per call, algorithmic bytes and FLOPs."""
+    from long_context_decode_c4a_b200 import ops
+    from synth.workloads import make_qpath_inputs
+    inp = make_qpath_inputs(M, device="cuda")
+    hidden, q_rank, H = inp["x"].shape[1], inp["wq_a"].shape[0], inp["wq_b"].shape[0] // 512
+    q = torch.empty(M, H, 512, dtype=torch.bfloat16, device="cuda")
+    ws = ops.workspace(ops._lib.CSA_WS_Q_PROJ, 1, 1, 1, 1, "cuda")
+    call = lambda: ops.q_projection(inp["x"], inp["wq_a"], inp["gamma_q"], inp["wq_b"], inp["pos"], H=H, q=q, ws=ws)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    if ops.device_status(ws) != 0:
+        raise RuntimeError("device status after the query path")
+    ms = e0.elapsed_time(e1) / steps
+    weights = (q_rank * hidden + H * 512 * q_rank) * 2
+    traffic = weights + M * hidden * 2 + 2 * M * q_rank * (4 + 2) + 2 * M * H * 512 * 2
+    flops = 2 * M * (q_rank * hidden + H * 512 * q_rank)
+    del inp, q
+    return ms, traffic, flops
+
+
 def extra_workloads(args, peaks):
     """Short measurements of the other synthetic configurations (one GPU, same process)."""
     res = {}
@@ -492,22 +521,27 @@ def extra_workloads(args, peaks):
                                   "frac": tf / peaks["bf16_tflops"], "flops_per_pass": attn_f + idx_f,
                                   "scope": "whole pass, algorithmic FLOPs (attention 4*H*reads*d + CSA indexer)"}}
         torch.cuda.empty_cache()
-    # The grouped output projection after the path ([P1] "输出投影也分组"): decode rows stream the
-    # 176 Mi weights (HBM-bound); prefill rows are a dense contraction (tensor-bound).
-    for name, M, steps in (("output_projection_decode_b64", 64, 20), ("output_projection_prefill_8k", 8192, 3)):
-        ms, traffic, flops = run_output_projection(M, steps, 3)
+    # The projections around the path: the low-rank query path before it ([P1] "低秩 Q", 106.5 Mi
+    # weights) and the grouped output projection after it ([P1] "输出投影也分组", 176 Mi). Decode rows
+    # stream the weights (HBM-bound); prefill rows are dense contractions (tensor-bound).
+    for name, M, steps, fn in (("q_path_decode_b64", 64, 20, run_q_path), ("q_path_prefill_8k", 8192, 3, run_q_path),
+                               ("output_projection_decode_b64", 64, 20, run_output_projection),
+                               ("output_projection_prefill_8k", 8192, 3, run_output_projection)):
+        ms, traffic, flops = fn(M, steps, 3)
         if M <= 256:
             ach = traffic / (ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": ach / peaks["hbm_gbs"], "bytes_per_call": traffic,
-                    "scope": "weights + o + r (written and read) + y, algorithmic bytes"}
+                    "scope": "weights + inputs + intermediates (written and read) + outputs, algorithmic bytes"}
         else:
             ach = flops / (ms * 1e-3) / 1e12
             roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": ach / peaks["bf16_tflops"], "flops_per_call": flops,
-                    "scope": "2*M*(G*R*Kg + D*G*R)"}
-        res[name] = {"value": M * 1000.0 / ms, "unit": "rows/s", "ms_per_step": ms, "rows": M,
-                     "shape": "G=16 groups x Kg=4096 -> R=1024, then 16384 -> D=7168", "roofline": roof}
+                    "scope": "2 x rows x weights (both contractions)"}
+        shape = ("hidden 7168 -> q_rank 1536 -> 128 heads x 512" if fn is run_q_path
+                 else "G=16 groups x Kg=4096 -> R=1024, then 16384 -> D=7168")
+        res[name] = {"value": M * 1000.0 / ms, "unit": "rows/s", "ms_per_step": ms, "rows": M, "shape": shape,
+                     "roofline": roof}
         torch.cuda.empty_cache()
     return res
 

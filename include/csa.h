@@ -84,7 +84,8 @@ enum {
   CSA_WS_HCA_ATTN = 3,
   CSA_WS_DECODE_FUSED = 4,
   CSA_WS_HCA_DECODE_FUSED = 5,
-  CSA_WS_OUTPUT_PROJ = 6
+  CSA_WS_OUTPUT_PROJ = 6,
+  CSA_WS_Q_PROJ = 7
 };
 
 /*
@@ -314,6 +315,39 @@ CSA_API int csa_indexer_topk_noalloc(int B, int S, int H_I, int d_I, int ratio, 
  */
 CSA_API int csa_output_projection(int M, int G, int Kg, int R, int D, const uint16_t* o, const uint16_t* wo_a,
                                   const uint16_t* wo_b, uint16_t* r, float* y, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/*
+ * csa_q_projection -- the low-rank query path in front of the layer ([P1] section "低秩 Q：两次
+ * 矩阵乘法接起来"), for M = B*S tokens:
+ *   qa = x . wq_a^T                        (fp32, written to the caller's scratch qa)
+ *   qr = gamma * qa / sqrt(mean(qa^2) + eps)   (bf16, written)
+ *   q  = qr . wq_b^T as [M, H, d], rounded to bf16, then each head divided by
+ *        sqrt(mean(q_h^2) + eps) and its last rope_dim dims rotated by pos[m]
+ *        (adjacent pairs, theta_i = rope_base^(-2i/rope_dim)); written as bf16.
+ *   x      dev bf16 [M, hidden].  wq_a: dev bf16 [q_rank, hidden].  gamma: dev bf16 [q_rank].
+ *   wq_b   dev bf16 [H*d, q_rank].  pos: dev int32 [M].
+ *   qa     dev float [M, q_rank] scratch.  qr: dev bf16 [M, q_rank].  q: dev bf16 [M, H, d].
+ *   ws/ws_bytes: workspace of at least csa_workspace_size(CSA_WS_Q_PROJ, ...) (status word).
+ * Supported: d = 512, rope_dim even and <= 128, hidden a multiple of 64, q_rank and H*d multiples
+ * of 128. Pro: hidden 7168, q_rank 1536, H 128. Alignment: pointers 16 bytes.
+ */
+CSA_API int csa_q_projection(int M, int hidden, int q_rank, int H, int d, int rope_dim, float rope_base, float eps,
+                             const int32_t* pos, const uint16_t* x, const uint16_t* wq_a, const uint16_t* gamma,
+                             const uint16_t* wq_b, float* qa, uint16_t* qr, uint16_t* q, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * csa_window_projection -- the window row of each token ([P5] §2: the KV down-projection
+ * [hidden] -> [head_dim], then RoPE on the last rope_dim dims; the pages' quantisation of the
+ * other dims is not applied): win[m] = RoPE_pos[m](x[m] . wkv^T), rounded to bf16 before the
+ * rotation and stored as bf16.
+ *   x dev bf16 [M, hidden]; wkv dev bf16 [d, hidden]; pos dev int32 [M]; win dev bf16 [M, d].
+ *   ws/ws_bytes: workspace of at least csa_workspace_size(CSA_WS_Q_PROJ, ...) (status word).
+ * Supported: d = 512, rope_dim even and <= 128, hidden a multiple of 64. Alignment: 16 bytes.
+ */
+CSA_API int csa_window_projection(int M, int hidden, int d, int rope_dim, float rope_base, const int32_t* pos,
+                                  const uint16_t* x, const uint16_t* wkv, uint16_t* win, void* ws, size_t ws_bytes,
                                   void* stream);
 
 /*

@@ -27,6 +27,7 @@ CSA_WS_HCA_ATTN = 3
 CSA_WS_DECODE_FUSED = 4
 CSA_WS_HCA_DECODE_FUSED = 5
 CSA_WS_OUTPUT_PROJ = 6
+CSA_WS_Q_PROJ = 7
 
 
 class CompressorCfg(ctypes.Structure):
@@ -89,6 +90,11 @@ PROTOTYPES = {
                                          c_void_p, c_int64, c_int, c_void_p, c_void_p]),
     "csa_output_projection": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p, c_void_p, c_size_t, c_void_p]),
+    "csa_q_projection": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_float, c_void_p, c_void_p,
+                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                 c_void_p]),
+    "csa_window_projection": (c_int, [c_int, c_int, c_int, c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p, c_size_t, c_void_p]),
 }
 
 _lib = None

@@ -440,6 +440,14 @@ int run_attn(const AttnArgs& a, bool csa_mode, cudaStream_t st) {
   return CSA_OK;
 }
 
+// K splits for a product whose output tiles alone would leave SMs idle: the largest power of two
+// (at most 8) that keeps every CTA in one wave and divides the K blocks.
+int gemm_splits(long long tiles, int kblocks, int sms) {
+  int splits = 1;
+  while (splits < 8 && tiles * splits * 2 <= sms && kblocks % (splits * 2) == 0) splits *= 2;
+  return splits;
+}
+
 // C = A . B^T on the tensor cores (gemm_kernel). A [a_rows, a_cols] and B [b_rows, b_cols] are
 // row-major bf16 with pitches lda / ldb; `groups` independent products along blockIdx.z.
 int run_gemm(const void* A, uint64_t a_cols, uint64_t a_rows, uint64_t lda, const void* Bm, uint64_t b_cols,
@@ -496,6 +504,7 @@ int csa_workspace_size(int kind, int B, int S, int max_entries, int topk, size_t
     case CSA_WS_HCA_ATTN:
     case CSA_WS_HCA_DECODE_FUSED:
     case CSA_WS_OUTPUT_PROJ:
+    case CSA_WS_Q_PROJ:
       *bytes = kStatusBytes;
       return CSA_OK;
     default:
@@ -588,10 +597,7 @@ int csa_output_projection(int M, int G, int Kg, int R, int D, const uint16_t* o,
                         (uint64_t)Kg, P1, G, dev->sms, st))
     return rc;
   // y = r . Wo_b^T; when the output tiles alone would leave SMs idle, K is split (fp32 reduction).
-  const long long tiles = (long long)(D / 128) * ((M + 127) / 128);
-  const int kblocks = G * R / 64;
-  int splits = 1;
-  while (splits < 8 && tiles * splits * 2 <= dev->sms && kblocks % (splits * 2) == 0) splits *= 2;
+  const int splits = gemm_splits((long long)(D / 128) * ((M + 127) / 128), G * R / 64, dev->sms);
   GemmParams P2{};
   P2.M = M;
   P2.N = D;
@@ -603,6 +609,109 @@ int csa_output_projection(int M, int G, int Kg, int R, int D, const uint16_t* o,
   P2.status = status;
   return run_gemm(r, (uint64_t)G * R, (uint64_t)M, (uint64_t)G * R, wo_b, (uint64_t)G * R, (uint64_t)D,
                   (uint64_t)G * R, P2, 1, dev->sms, st);
+}
+
+int csa_q_projection(int M, int hidden, int q_rank, int H, int d, int rope_dim, float rope_base, float eps,
+                     const int32_t* pos, const uint16_t* x, const uint16_t* wq_a, const uint16_t* gamma,
+                     const uint16_t* wq_b, float* qa, uint16_t* qr, uint16_t* q, void* ws, size_t ws_bytes,
+                     void* stream) {
+  CSA_CHECK_ARG(M > 0 && hidden > 0 && q_rank > 0 && H > 0, "sizes must be positive");
+  CSA_CHECK_ARG(pos && x && wq_a && gamma && wq_b && qa && qr && q, "null pointer");
+  CSA_CHECK_ARG(aligned(x, 16) && aligned(wq_a, 16) && aligned(gamma, 16) && aligned(wq_b, 16) && aligned(qa, 16) &&
+                    aligned(qr, 16) && aligned(q, 16) && aligned(pos, 4),
+                "pointers must be 16-byte aligned");
+  CSA_CHECK_SUP(d == 512, "d must be 512");
+  CSA_CHECK_SUP(rope_dim > 0 && rope_dim % 2 == 0 && rope_dim / 2 <= kMaxRopePairs, "rope_dim must be even, <= 128");
+  CSA_CHECK_SUP(hidden % 64 == 0 && q_rank % 128 == 0 && (H * d) % 128 == 0,
+                "hidden must be a multiple of 64, q_rank and H*d of 128");
+  CSA_CHECK_SUP((long long)M * H <= (1LL << 31) - 1, "too many rows");
+  if (int rc = check_ws(ws, ws_bytes, kStatusBytes)) return rc;
+  DeviceInfo* dev;
+  if (int rc = device_info(&dev)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  // qa = x . wq_a^T (fp32; split over K when the 128-column tiles alone leave SMs idle).
+  GemmParams P1{};
+  P1.M = M;
+  P1.N = q_rank;
+  P1.K = hidden;
+  P1.splits = gemm_splits((long long)(q_rank / 128) * ((M + 127) / 128), hidden / 64, dev->sms);
+  P1.ldc = q_rank;
+  P1.c = qa;
+  P1.c_mode = P1.splits > 1 ? kGemmOutF32Add : kGemmOutF32;
+  P1.status = status;
+  if (int rc = run_gemm(x, (uint64_t)hidden, (uint64_t)M, (uint64_t)hidden, wq_a, (uint64_t)hidden, (uint64_t)q_rank,
+                        (uint64_t)hidden, P1, 1, dev->sms, st))
+    return rc;
+  CSA_CUDA(launch_pdl(rmsnorm_rows_kernel, dim3((unsigned)M), dim3(kRowNormThreads), 0, st,
+                      static_cast<const float*>(qa), gamma, qr, q_rank, eps));
+  // q = qr . wq_b^T (bf16), then the per-head norm and RoPE in place.
+  GemmParams P2{};
+  P2.M = M;
+  P2.N = H * d;
+  P2.K = q_rank;
+  P2.splits = 1;
+  P2.ldc = (long long)H * d;
+  P2.c = q;
+  P2.c_mode = kGemmOutBf16;
+  P2.status = status;
+  if (int rc = run_gemm(qr, (uint64_t)q_rank, (uint64_t)M, (uint64_t)q_rank, wq_b, (uint64_t)q_rank,
+                        (uint64_t)H * d, (uint64_t)q_rank, P2, 1, dev->sms, st))
+    return rc;
+  HeadNormParams N{};
+  N.M = M;
+  N.H = H;
+  N.rope_dim = rope_dim;
+  N.normalize = 1;
+  N.eps = eps;
+  for (int i = 0; i < rope_dim / 2; ++i) N.inv_freq[i] = std::pow((double)rope_base, -2.0 * i / rope_dim);
+  N.pos = pos;
+  N.q = q;
+  const long long items = (long long)M * H;
+  const int per = kHeadNormThreads / 32;
+  CSA_CUDA(launch_pdl(head_norm_rope_kernel, dim3((unsigned)((items + per - 1) / per)), dim3(kHeadNormThreads), 0,
+                      st, N));
+  return CSA_OK;
+}
+
+int csa_window_projection(int M, int hidden, int d, int rope_dim, float rope_base, const int32_t* pos,
+                          const uint16_t* x, const uint16_t* wkv, uint16_t* win, void* ws, size_t ws_bytes,
+                          void* stream) {
+  CSA_CHECK_ARG(M > 0 && hidden > 0, "sizes must be positive");
+  CSA_CHECK_ARG(pos && x && wkv && win, "null pointer");
+  CSA_CHECK_ARG(aligned(x, 16) && aligned(wkv, 16) && aligned(win, 16) && aligned(pos, 4),
+                "pointers must be 16-byte aligned");
+  CSA_CHECK_SUP(d == 512, "d must be 512");
+  CSA_CHECK_SUP(rope_dim > 0 && rope_dim % 2 == 0 && rope_dim / 2 <= kMaxRopePairs, "rope_dim must be even, <= 128");
+  CSA_CHECK_SUP(hidden % 64 == 0, "hidden must be a multiple of 64");
+  if (int rc = check_ws(ws, ws_bytes, kStatusBytes)) return rc;
+  DeviceInfo* dev;
+  if (int rc = device_info(&dev)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  GemmParams P{};
+  P.M = M;
+  P.N = d;
+  P.K = hidden;
+  P.splits = 1;
+  P.ldc = d;
+  P.c = win;
+  P.c_mode = kGemmOutBf16;
+  P.status = reinterpret_cast<uint32_t*>(ws);
+  if (int rc = run_gemm(x, (uint64_t)hidden, (uint64_t)M, (uint64_t)hidden, wkv, (uint64_t)hidden, (uint64_t)d,
+                        (uint64_t)hidden, P, 1, dev->sms, st))
+    return rc;
+  HeadNormParams N{};
+  N.M = M;
+  N.H = 1;
+  N.rope_dim = rope_dim;
+  N.normalize = 0;
+  N.eps = 0.f;
+  for (int i = 0; i < rope_dim / 2; ++i) N.inv_freq[i] = std::pow((double)rope_base, -2.0 * i / rope_dim);
+  N.pos = pos;
+  N.q = win;
+  const int per = kHeadNormThreads / 32;
+  CSA_CUDA(launch_pdl(head_norm_rope_kernel, dim3((unsigned)((M + per - 1) / per)), dim3(kHeadNormThreads), 0, st, N));
+  return CSA_OK;
 }
 
 int csa_decode_fused(const csa_decode_args* a, void* stream) {

@@ -153,6 +153,23 @@ __global__ void gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __g
                             GemmParams P);
 __global__ void zero_f32_kernel(float* p, long long n4);
 
+// ------------------------------------------------------------------------------ query path
+
+constexpr int kRowNormThreads = 256;
+constexpr int kHeadNormThreads = 256;     // 8 warps: one (row, head) each
+
+struct HeadNormParams {
+  int M, H, rope_dim;
+  int normalize;                          // 1: divide each head by its RMS first (query path)
+  float eps;
+  double inv_freq[kMaxRopePairs];         // rope_base^(-2i/rope_dim), formed on the host in double
+  const int32_t* pos;                     // [M] token positions
+  uint16_t* q;                            // [M, H, 512] bf16, normalised and rotated in place
+};
+
+__global__ void rmsnorm_rows_kernel(const float* x, const uint16_t* gamma, uint16_t* y, int n, float eps);
+__global__ void head_norm_rope_kernel(HeadNormParams P);
+
 size_t attn_smem_bytes();
 size_t gemm_smem_bytes();
 size_t indexer_smem_bytes(int stages, int N);

@@ -382,6 +382,52 @@ def output_projection(o: torch.Tensor, wo_a: torch.Tensor, wo_b: torch.Tensor, r
     return r, y
 
 
+def q_projection(x: torch.Tensor, wq_a: torch.Tensor, gamma: torch.Tensor, wq_b: torch.Tensor, pos: torch.Tensor,
+                 H: int = 128, d: int = 512, rope_dim: int = 64, rope_base: float = 10000.0, eps: float = 1e-6,
+                 q: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """Low-rank query path: x [M, hidden], wq_a [q_rank, hidden], gamma [q_rank], wq_b [H*d, q_rank]
+    (bf16), pos [M] int32. Returns (qa fp32 [M, q_rank], qr bf16 [M, q_rank], q bf16 [M, H, d])."""
+    M, hidden = x.shape
+    q_rank = wq_a.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(wq_a, "wq_a", torch.bfloat16, (q_rank, hidden))
+    _need(gamma, "gamma", torch.bfloat16, (q_rank,))
+    _need(wq_b, "wq_b", torch.bfloat16, (H * d, q_rank))
+    _need(pos, "pos", torch.int32, (M,))
+    qa = torch.empty(M, q_rank, dtype=torch.float32, device=x.device)
+    qr = torch.empty(M, q_rank, dtype=torch.bfloat16, device=x.device)
+    if q is None:
+        q = torch.empty(M, H, d, dtype=torch.bfloat16, device=x.device)
+    _need(q, "q", torch.bfloat16, (M, H, d))
+    if ws is None:
+        ws = workspace(_lib.CSA_WS_Q_PROJ, 1, 1, 1, 1, x.device)
+    check(_lib.load().csa_q_projection(M, hidden, q_rank, H, d, rope_dim, rope_base, eps, pos.data_ptr(),
+                                       x.data_ptr(), wq_a.data_ptr(), gamma.data_ptr(), wq_b.data_ptr(),
+                                       qa.data_ptr(), qr.data_ptr(), q.data_ptr(), ws.data_ptr(), ws.numel(),
+                                       _stream()), "csa_q_projection")
+    return qa, qr, q
+
+
+def window_projection(x: torch.Tensor, wkv: torch.Tensor, pos: torch.Tensor, rope_dim: int = 64,
+                      rope_base: float = 10000.0, win: Optional[torch.Tensor] = None,
+                      ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Window rows: RoPE_pos(x . wkv^T) for x [M, hidden], wkv [d, hidden] bf16; returns bf16 [M, d]."""
+    M, hidden = x.shape
+    d = wkv.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(wkv, "wkv", torch.bfloat16, (d, hidden))
+    _need(pos, "pos", torch.int32, (M,))
+    if win is None:
+        win = torch.empty(M, d, dtype=torch.bfloat16, device=x.device)
+    _need(win, "win", torch.bfloat16, (M, d))
+    if ws is None:
+        ws = workspace(_lib.CSA_WS_Q_PROJ, 1, 1, 1, 1, x.device)
+    check(_lib.load().csa_window_projection(M, hidden, d, rope_dim, rope_base, pos.data_ptr(), x.data_ptr(),
+                                            wkv.data_ptr(), win.data_ptr(), ws.data_ptr(), ws.numel(), _stream()),
+          "csa_window_projection")
+    return win
+
+
 def device_status(ws: torch.Tensor) -> int:
     """Synchronise the current stream, read and clear the workspace's device status word."""
     st = ctypes.c_int(0)

@@ -35,6 +35,9 @@ Where the pages are silent the oracle takes one reading, named READING-n below:
   R14 the compressor scores are used as given (no extra bias).
   R20 output projection: the intermediate r of each group is rounded to bf16 before the second
       product (the pages give the two einsums, not the precision between them).
+  R21 query path: qr = rms_norm(x Wq_a^T) uses a weight gamma and eps = 1e-6 (as R3) and is rounded
+      to bf16 before the second product; the product qr Wq_b^T is rounded to bf16 before the
+      per-head norm; the window row x Wkv^T is rounded to bf16 before its rotation.
 """
 
 from __future__ import annotations
@@ -318,6 +321,32 @@ def output_projection(o_rows: np.ndarray, wo_a: np.ndarray, wo_b: np.ndarray):
     rb = bf16(r)
     y = rb.reshape(M, G * R) @ wo_b.T
     return r.reshape(M, G * R), rb.reshape(M, G * R), y
+
+
+# ----------------------------------------------------------------------------- query path
+
+def q_path(x: np.ndarray, wq_a: np.ndarray, gamma: np.ndarray, wq_b: np.ndarray, pos: np.ndarray, H: int,
+           d: int = 512, rope_dim: int = 64, rope_base: float = 10000.0, eps: float = 1e-6):
+    """[P1] "低秩 Q：两次矩阵乘法接起来": qr = rms_norm(x Wq_a^T); q = (qr Wq_b^T) as [M, H, d];
+    q = q / sqrt(mean(q^2 over each head) + eps) (no weight); the last rope_dim dims of each head are
+    rotated by the token's position. Precision per R21. Returns (qa, qr rounded to bf16, q)."""
+    M = x.shape[0]
+    qa = x @ wq_a.T
+    qr = bf16(rms_norm(qa, gamma, eps))
+    qraw = bf16(qr @ wq_b.T).reshape(M, H, d)
+    q = qraw / np.sqrt(np.mean(qraw * qraw, axis=-1, keepdims=True) + eps)
+    for m in range(M):
+        q[m] = rope(q[m], float(pos[m]), rope_dim, rope_base)
+    return qa, qr, q
+
+
+def window_projection(x: np.ndarray, wkv: np.ndarray, pos: np.ndarray, rope_dim: int = 64,
+                      rope_base: float = 10000.0) -> np.ndarray:
+    """[P5] §2: the window row of each token is its KV down-projection x Wkv^T ([hidden] -> [d]) with
+    the last rope_dim dims rotated by the token's position (R21: rounded to bf16 first; the pages'
+    quantisation of the other dims is not applied, R16)."""
+    w = bf16(x @ wkv.T)
+    return np.stack([rope(w[m], float(pos[m]), rope_dim, rope_base) for m in range(x.shape[0])])
 
 
 # ----------------------------------------------------------------------------- counters

@@ -200,3 +200,24 @@ def make_oproj_inputs(M: int, G: int = OPROJ_GROUPS, Kg: int = OPROJ_KG, R: int 
     wa = _randn(gen, (G, R, Kg), device, dtype=torch.float32).mul_(1.0 / math.sqrt(Kg)).to(torch.bfloat16)
     wb = _randn(gen, (D, G * R), device, dtype=torch.float32).mul_(1.0 / math.sqrt(G * R)).to(torch.bfloat16)
     return {"o": o, "wo_a": wa, "wo_b": wb}
+
+
+# Low-rank query path ([P1] "低秩 Q") and the window-row projection: Pro shapes.
+QPATH_HIDDEN, QPATH_RANK, QPATH_HEADS = 7168, 1536, 128
+
+
+def make_qpath_inputs(M: int, hidden: int = QPATH_HIDDEN, q_rank: int = QPATH_RANK, H: int = QPATH_HEADS,
+                      d: int = 512, start_pos: int = 0, seed: int = 0, device: str = "cpu") -> Dict[str, torch.Tensor]:
+    """Seeded inputs of the query path and the window-row projection: x [M, hidden] ~ bf16 N(0,1),
+    Wq_a [q_rank, hidden] ~ N(0,1)/sqrt(hidden), gamma = 1, Wq_b [H*d, q_rank] ~ N(0,1)/sqrt(q_rank),
+    Wkv [d, hidden] ~ N(0,1)/sqrt(hidden) (bf16), positions start_pos .. start_pos+M-1.
+    Draw order: x, Wq_a, Wq_b, Wkv."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    x = _randn(gen, (M, hidden), device)
+    wa = _randn(gen, (q_rank, hidden), device, dtype=torch.float32).mul_(1.0 / math.sqrt(hidden)).to(torch.bfloat16)
+    wb = _randn(gen, (H * d, q_rank), device, dtype=torch.float32).mul_(1.0 / math.sqrt(q_rank)).to(torch.bfloat16)
+    wkv = _randn(gen, (d, hidden), device, dtype=torch.float32).mul_(1.0 / math.sqrt(hidden)).to(torch.bfloat16)
+    pos = torch.arange(start_pos, start_pos + M, dtype=torch.int32, device=device)
+    return {"x": x, "wq_a": wa, "gamma_q": torch.ones(q_rank, dtype=torch.bfloat16, device=device), "wq_b": wb,
+            "wkv": wkv, "pos": pos}

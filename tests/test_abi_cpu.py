@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     names = declared_symbols()
     for want in ("csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode_fused",
                  "hca_decode_fused", "csa_workspace_size", "csa_get_device_status", "csa_state_reset",
-                 "csa_output_projection"):
+                 "csa_output_projection", "csa_q_projection", "csa_window_projection"):
         assert want in names
 
 
@@ -139,4 +139,14 @@ def test_host_side_argument_checks_launch_nothing(lib):
         _lib.CSA_ERR_UNSUPPORTED
     assert lib.csa_output_projection(64, 16, 4096, 1024, 7168, 16, 16, 16, 16, 16, null, 0, null) == \
         _lib.CSA_ERR_WORKSPACE
+    # query path / window rows: d must be 512, q_rank a multiple of 128, pointers present
+    assert lib.csa_q_projection(64, 7168, 1536, 128, 256, 64, 1e4, 1e-6, 16, 16, 16, 16, 16, 16, 16, 16, 256, 256,
+                                null) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_q_projection(64, 7168, 1500, 128, 512, 64, 1e4, 1e-6, 16, 16, 16, 16, 16, 16, 16, 16, 256, 256,
+                                null) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_q_projection(64, 7168, 1536, 128, 512, 64, 1e4, 1e-6, null, 16, 16, 16, 16, 16, 16, 16, 256, 256,
+                                null) == _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_window_projection(64, 7168, 512, 63, 1e4, 16, 16, 16, 16, 256, 256, null) == \
+        _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_window_projection(64, 7168, 512, 64, 1e4, 16, 16, 16, 16, null, 0, null) == _lib.CSA_ERR_WORKSPACE
     assert lib.csa_last_error()

@@ -426,3 +426,58 @@ def test_output_projection_groups_are_independent_and_linear():
     for g in range(G):
         assert np.allclose(r[:, g * R:(g + 1) * R], o[:, g * Kg:(g + 1) * Kg] @ wa[g].T, rtol=1e-14, atol=1e-12)
     assert np.array_equal(rb, O.bf16(r))
+
+
+# ----------------------------------------------------------------------------- query path
+
+def _complex_rotate(v, pos, rope_dim, base):
+    """Rotation of the last rope_dim dims as complex multiplication (textbook form)."""
+    head = v.shape[-1] - rope_dim
+    z = v[..., head::2] + 1j * v[..., head + 1::2]
+    theta = base ** (-np.arange(rope_dim // 2) * 2.0 / rope_dim)
+    z = z * np.exp(1j * pos * theta)
+    out = v.copy()
+    out[..., head::2] = z.real
+    out[..., head + 1::2] = z.imag
+    return out
+
+
+def test_q_path_one_hot_weights_closed_form():
+    """[P1] "低秩 Q": with Wq_a selecting input dims and Wq_b selecting qr dims, every step has a closed
+    form: qa = selected x, qr = gamma qa / sqrt(mean(qa^2) + eps), each head of q = its selected qr
+    values over their RMS, then the complex rotation of its last 64 dims by the position."""
+    rng = np.random.default_rng(30)
+    M, hidden, q_rank, H, d, eps = 3, 64, 16, 2, 512, 1e-6
+    x = O.bf16(rng.standard_normal((M, hidden)))
+    sel_a = rng.choice(hidden, q_rank, replace=False)
+    wq_a = np.zeros((q_rank, hidden))
+    wq_a[np.arange(q_rank), sel_a] = 1.0
+    gamma = O.bf16(rng.uniform(0.5, 1.5, q_rank))
+    sel_b = rng.integers(0, q_rank, H * d)
+    wq_b = np.zeros((H * d, q_rank))
+    wq_b[np.arange(H * d), sel_b] = 1.0
+    pos = np.array([0, 7, 123456])
+    qa, qr, q = O.q_path(x, wq_a, gamma, wq_b, pos, H, d, eps=eps)
+    assert np.array_equal(qa, x[:, sel_a])
+    exp_qr = O.bf16(gamma * x[:, sel_a] / np.sqrt(np.mean(x[:, sel_a] ** 2, axis=1, keepdims=True) + eps))
+    assert np.array_equal(qr, exp_qr)
+    for m in range(M):
+        heads = exp_qr[m, sel_b].reshape(H, d)
+        heads = heads / np.sqrt(np.mean(heads ** 2, axis=1, keepdims=True) + eps)
+        assert np.allclose(q[m], _complex_rotate(heads, pos[m], 64, 10000.0), rtol=0, atol=1e-12)
+    # position 0 leaves q unrotated; every head keeps its mean square m / (m + eps)
+    assert np.allclose(np.mean(q ** 2, axis=-1), 1.0, atol=1e-4)
+
+
+def test_window_projection_one_hot_closed_form():
+    """[P5] §2: the window row is the down-projected row with its last 64 dims rotated by the position."""
+    rng = np.random.default_rng(31)
+    M, hidden, d = 2, 1024, 512
+    x = O.bf16(rng.standard_normal((M, hidden)))
+    sel = rng.choice(hidden, d, replace=False)
+    wkv = np.zeros((d, hidden))
+    wkv[np.arange(d), sel] = 1.0
+    pos = np.array([5, 99999])
+    w = O.window_projection(x, wkv, pos)
+    for m in range(M):
+        assert np.allclose(w[m], _complex_rotate(x[m, sel], pos[m], 64, 10000.0), rtol=0, atol=1e-12)
