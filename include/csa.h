@@ -144,7 +144,7 @@ CSA_API int csa_compress(const csa_compressor_cfg* cfg, int B, int S, const int3
  *   topk_idx  dev int32 [B, S, topk], out.
  *   scores_opt optional dev float [B, S, max_entries], out (nullable): the scores, s < E only.
  *   ws/ws_bytes: workspace of at least csa_workspace_size(CSA_WS_INDEXER_TOPK, ...).
- * Supported: d_I = 128; H_I a power of two <= 256; topk in [1, 2048]; E <= max_entries <= 2^24.
+ * Supported: d_I = 128; H_I a power of two in [4, 128]; topk in [1, 2048]; E <= max_entries <= 2^24.
  * A query with E > max_entries records CSA_ERR_BOUNDS in the status word and uses max_entries.
  */
 CSA_API int csa_indexer_topk(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
@@ -278,6 +278,23 @@ typedef struct {
 
 /* hca_decode_fused -- one HCA decode step ([P5] §3): C128A step, window write, hca_attn. */
 CSA_API int hca_decode_fused(const hca_decode_args* a, void* stream);
+
+/*
+ * csa_indexer_scores / csa_topk -- the two halves of csa_indexer_topk, for the tensor-parallel
+ * indexer ([P1] "少读 KV 之前，Indexer 仍要给历史打分": with the indexer heads split over ranks, the
+ * partial scores are summed across ranks before the selection). csa_indexer_scores writes
+ * scores[b, i, s] = sum over this call's H_I heads of w[h] * ReLU(q_idx[h,:] . idx_cache[s,:]) for the
+ * visible s < E (entries s >= E are not written); its workspace holds only the status word
+ * (csa_workspace_size(CSA_WS_SPARSE_ATTN, ...) suffices). csa_topk selects, from caller-provided
+ * scores [B, S, max_entries], exactly as csa_indexer_topk does; its workspace:
+ * csa_workspace_size(CSA_WS_INDEXER_TOPK, ...) (an upper bound). Arguments, layouts and limits as
+ * in csa_indexer_topk; scores must be 16-byte aligned.
+ */
+CSA_API int csa_indexer_scores(int B, int S, int H_I, int d_I, int ratio, const int32_t* q_pos, const uint16_t* q_idx,
+                               const float* w, const uint16_t* idx_cache, int64_t idx_bstride, int max_entries,
+                               float* scores, void* ws, size_t ws_bytes, void* stream);
+CSA_API int csa_topk(int B, int S, int ratio, int topk, const int32_t* q_pos, const float* scores, int max_entries,
+                     int32_t* topk_idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * csa_indexer_topk_noalloc -- csa_indexer_topk for callers that cannot allocate device memory (no

@@ -252,15 +252,24 @@ struct IndexerArgs {
   size_t ws_bytes;
 };
 
-int check_indexer_args(const IndexerArgs& a) {
+int check_indexer_args(const IndexerArgs& a, bool scores = true, bool select = true) {
   CSA_CHECK_ARG(a.B > 0 && a.S > 0, "B and S must be positive");
+  if (!scores) {  // selection over caller-provided scores
+    CSA_CHECK_ARG(a.ratio > 0, "ratio must be positive");
+    CSA_CHECK_SUP(a.topk >= 1 && a.topk <= kAttnMaxTopk, "topk must be in [1, %d]", kAttnMaxTopk);
+    CSA_CHECK_SUP(a.max_entries >= 1 && a.max_entries <= (1 << 24), "max_entries must be in [1, 2^24]");
+    CSA_CHECK_ARG(a.q_pos && a.scores_opt && a.topk_idx, "null pointer argument");
+    CSA_CHECK_ARG(aligned(a.scores_opt, 16) && aligned(a.topk_idx, 4) && aligned(a.q_pos, 4), "misaligned pointer");
+    return CSA_OK;
+  }
+  if (!select) CSA_CHECK_ARG(a.scores_opt != nullptr, "scores is null");
   CSA_CHECK_SUP(a.d_I == 128, "d_I must be 128");
   CSA_CHECK_SUP(a.H_I == 4 || a.H_I == 8 || a.H_I == 16 || a.H_I == 32 || a.H_I == 64 || a.H_I == 128,
                 "H_I must be a power of two in [4, 128]");
   CSA_CHECK_ARG(a.ratio > 0, "ratio must be positive");
   CSA_CHECK_SUP(a.topk >= 1 && a.topk <= kAttnMaxTopk, "topk must be in [1, %d]", kAttnMaxTopk);
   CSA_CHECK_SUP(a.max_entries >= 1 && a.max_entries <= (1 << 24), "max_entries must be in [1, 2^24]");
-  CSA_CHECK_ARG(a.q_pos && a.q_idx && a.w && a.idx_cache && a.topk_idx, "null pointer argument");
+  CSA_CHECK_ARG(a.q_pos && a.q_idx && a.w && a.idx_cache && (a.topk_idx || !select), "null pointer argument");
   CSA_CHECK_ARG(aligned(a.q_idx, 16) && aligned(a.idx_cache, 16) && aligned(a.w, 4) && aligned(a.topk_idx, 4) &&
                     aligned(a.q_pos, 4),
                 "misaligned pointer");
@@ -274,57 +283,67 @@ int check_indexer_args(const IndexerArgs& a) {
   return CSA_OK;
 }
 
-int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* ev = nullptr) {
+// The indexer (scores) and / or the top-k selection over them. Scores-only and selection-only calls
+// serve the tensor-parallel indexer: partial scores per head shard, a sum across ranks, then the
+// selection.
+int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* ev = nullptr, bool run_scores = true,
+                     bool run_select = true) {
   DeviceInfo* dev;
   if (int rc = device_info(&dev)) return rc;
   const long long queries = (long long)a.B * a.S;
-  const IdxWs L = indexer_ws_layout(queries, a.max_entries, a.topk);
-  if (int rc = check_ws(a.ws, a.ws_bytes, L.total)) return rc;
+  const IdxWs L = indexer_ws_layout(queries, a.max_entries, run_select ? a.topk : 1);
+  const size_t need = run_select ? (a.scores_opt ? L.total - (L.cand_key_off - L.scores_off) : L.total) : kStatusBytes;
+  if (int rc = check_ws(a.ws, a.ws_bytes, need)) return rc;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  // With caller-provided scores the workspace's score region is not needed: the candidate lists
+  // move down to start right after the status word.
+  const size_t shift = a.scores_opt ? (L.cand_key_off - L.scores_off) : 0;
   float* scores = a.scores_opt ? a.scores_opt : reinterpret_cast<float*>(ws + L.scores_off);
+  if (run_scores) {
+    IndexerParams P{};
+    P.B = a.B;
+    P.S = a.S;
+    P.QG = a.S == 1 ? 1 : std::min(a.S, 256 / a.H_I);
+    P.N = (int)round_up((size_t)P.QG * a.H_I, 16);
+    P.ratio = a.ratio;
+    P.max_entries = a.max_entries;
+    P.groups_per_req = (a.S + P.QG - 1) / P.QG;
+    P.tiles_per_group = (a.max_entries + 127) / 128;
+    P.total_items = (long long)a.B * P.groups_per_req * P.tiles_per_group;
+    P.rows_per_req = a.idx_bstride / a.d_I;
+    int stages = kIdxMaxStages;
+    while (stages > 2 && indexer_smem_bytes(stages, P.N) > (size_t)dev->max_smem) --stages;
+    CSA_CHECK_SUP(indexer_smem_bytes(stages, P.N) <= (size_t)dev->max_smem, "shared memory too small for the indexer");
+    P.stages = stages;
+    P.n_acc = (4 * P.N <= 512) ? 4 : 2;
+    int cols = 32;
+    while (cols < P.n_acc * P.N) cols <<= 1;
+    P.tmem_cols = cols;
+    P.q_pos = a.q_pos;
+    P.w = a.w;
+    P.scores = scores;
+    P.scores_stride = a.max_entries;
+    P.status = status;
 
-  IndexerParams P{};
-  P.B = a.B;
-  P.S = a.S;
-  P.QG = a.S == 1 ? 1 : std::min(a.S, 256 / a.H_I);
-  P.N = (int)round_up((size_t)P.QG * a.H_I, 16);
-  P.ratio = a.ratio;
-  P.max_entries = a.max_entries;
-  P.groups_per_req = (a.S + P.QG - 1) / P.QG;
-  P.tiles_per_group = (a.max_entries + 127) / 128;
-  P.total_items = (long long)a.B * P.groups_per_req * P.tiles_per_group;
-  P.rows_per_req = a.idx_bstride / a.d_I;
-  int stages = kIdxMaxStages;
-  while (stages > 2 && indexer_smem_bytes(stages, P.N) > (size_t)dev->max_smem) --stages;
-  CSA_CHECK_SUP(indexer_smem_bytes(stages, P.N) <= (size_t)dev->max_smem, "shared memory too small for the indexer");
-  P.stages = stages;
-  P.n_acc = (4 * P.N <= 512) ? 4 : 2;
-  int cols = 32;
-  while (cols < P.n_acc * P.N) cols <<= 1;
-  P.tmem_cols = cols;
-  P.q_pos = a.q_pos;
-  P.w = a.w;
-  P.scores = scores;
-  P.scores_stride = a.max_entries;
-  P.status = status;
-
-  CUtensorMap map_k, map_q;
-  if (int rc = make_map_2d(&map_k, a.idx_cache, 128, (uint64_t)a.B * P.rows_per_req, 128, 64, 128)) return rc;
-  if (int rc = make_map_2d(&map_q, a.q_idx, 128, (uint64_t)queries * a.H_I, 128, 64, (uint32_t)P.N)) return rc;
-  const size_t smem = indexer_smem_bytes(stages, P.N);
-  const dim3 grid((unsigned)std::min<long long>(P.total_items, dev->sms));
-  cudaError_t e = cudaSuccess;
-  switch (a.H_I) {
-    case 4: e = launch_pdl(indexer_kernel<4>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-    case 8: e = launch_pdl(indexer_kernel<8>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-    case 16: e = launch_pdl(indexer_kernel<16>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-    case 32: e = launch_pdl(indexer_kernel<32>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-    case 64: e = launch_pdl(indexer_kernel<64>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-    default: e = launch_pdl(indexer_kernel<128>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+    CUtensorMap map_k, map_q;
+    if (int rc = make_map_2d(&map_k, a.idx_cache, 128, (uint64_t)a.B * P.rows_per_req, 128, 64, 128)) return rc;
+    if (int rc = make_map_2d(&map_q, a.q_idx, 128, (uint64_t)queries * a.H_I, 128, 64, (uint32_t)P.N)) return rc;
+    const size_t smem = indexer_smem_bytes(stages, P.N);
+    const dim3 grid((unsigned)std::min<long long>(P.total_items, dev->sms));
+    cudaError_t e = cudaSuccess;
+    switch (a.H_I) {
+      case 4: e = launch_pdl(indexer_kernel<4>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+      case 8: e = launch_pdl(indexer_kernel<8>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+      case 16: e = launch_pdl(indexer_kernel<16>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+      case 32: e = launch_pdl(indexer_kernel<32>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+      case 64: e = launch_pdl(indexer_kernel<64>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+      default: e = launch_pdl(indexer_kernel<128>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+    }
+    CSA_CUDA(e);
   }
-  CSA_CUDA(e);
   if (ev) CSA_CUDA(cudaEventRecord(ev[0], st));
+  if (!run_select) return CSA_OK;
 
   TopkParams T{};
   T.topk = a.topk;
@@ -336,9 +355,9 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
   T.scores = scores;
   T.scores_stride = a.max_entries;
   T.out = a.topk_idx;
-  T.cand_key = reinterpret_cast<uint32_t*>(ws + L.cand_key_off);
-  T.cand_idx = reinterpret_cast<int32_t*>(ws + L.cand_idx_off);
-  T.cand_cnt = reinterpret_cast<int*>(ws + L.cand_cnt_off);
+  T.cand_key = reinterpret_cast<uint32_t*>(ws + L.cand_key_off - shift);
+  T.cand_idx = reinterpret_cast<int32_t*>(ws + L.cand_idx_off - shift);
+  T.cand_cnt = reinterpret_cast<int*>(ws + L.cand_cnt_off - shift);
   T.status = status;
   const int nchunks = std::max(1, L.max_chunks);
   const int tk_threads = a.max_entries <= kTopkShortRow ? kTopkShortThreads : kTopkThreads;
@@ -533,6 +552,23 @@ int csa_compress(const csa_compressor_cfg* cfg, int B, int S, const int32_t* sta
                            max_entries, cache_f32, nullptr);
   L.p[1] = L.p[0];
   return launch_compress(L, 1, B, S, cfg->ratio, static_cast<cudaStream_t>(stream));
+}
+
+int csa_indexer_scores(int B, int S, int H_I, int d_I, int ratio, const int32_t* q_pos, const uint16_t* q_idx,
+                       const float* w, const uint16_t* idx_cache, int64_t idx_bstride, int max_entries, float* scores,
+                       void* ws, size_t ws_bytes, void* stream) {
+  IndexerArgs a{B, S, H_I, d_I, ratio, 1, q_pos, q_idx, w, idx_cache, idx_bstride, max_entries, nullptr, scores,
+                ws, ws_bytes};
+  if (int rc = check_indexer_args(a, true, false)) return rc;
+  return run_indexer_topk(a, static_cast<cudaStream_t>(stream), nullptr, true, false);
+}
+
+int csa_topk(int B, int S, int ratio, int topk, const int32_t* q_pos, const float* scores, int max_entries,
+             int32_t* topk_idx, void* ws, size_t ws_bytes, void* stream) {
+  IndexerArgs a{B, S, 0, 0, ratio, topk, q_pos, nullptr, nullptr, nullptr, 0, max_entries, topk_idx,
+                const_cast<float*>(scores), ws, ws_bytes};
+  if (int rc = check_indexer_args(a, false, true)) return rc;
+  return run_indexer_topk(a, static_cast<cudaStream_t>(stream), nullptr, false, true);
 }
 
 int csa_indexer_topk(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,

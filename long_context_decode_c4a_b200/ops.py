@@ -116,6 +116,44 @@ def indexer_topk(q_pos: torch.Tensor, q_idx: torch.Tensor, w: torch.Tensor, idx_
     return topk_idx
 
 
+def indexer_scores(q_pos: torch.Tensor, q_idx: torch.Tensor, w: torch.Tensor, idx_cache: torch.Tensor,
+                   ratio: int = 4, scores: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None
+                   ) -> torch.Tensor:
+    """Indexer scores over this call's heads only (no selection): scores [B,S,max_entries] fp32, the
+    visible s < (t+1)//ratio written. With the heads split over ranks, these are partial scores."""
+    B, S, H_I, d_I = q_idx.shape
+    E = idx_cache.shape[1]
+    _need(q_pos, "q_pos", torch.int32, (B, S))
+    _need(q_idx, "q_idx", torch.bfloat16)
+    _need(w, "w", torch.float32, (B, S, H_I))
+    if scores is None:
+        scores = torch.empty(B, S, E, dtype=torch.float32, device=q_idx.device)
+    _need(scores, "scores", torch.float32, (B, S, E))
+    if ws is None:
+        ws = workspace(_lib.CSA_WS_SPARSE_ATTN, B, S, E, 1, q_idx.device)
+    check(_lib.load().csa_indexer_scores(B, S, H_I, d_I, ratio, q_pos.data_ptr(), q_idx.data_ptr(), w.data_ptr(),
+                                         idx_cache.data_ptr(), _bstride(idx_cache, "idx_cache"), E, scores.data_ptr(),
+                                         ws.data_ptr(), ws.numel(), _stream()), "csa_indexer_scores")
+    return scores
+
+
+def topk(q_pos: torch.Tensor, scores: torch.Tensor, k: int, ratio: int = 4, topk_idx: Optional[torch.Tensor] = None,
+         ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The selection of csa_indexer_topk over given scores [B,S,max_entries] fp32: the min(k, E)
+    largest of the visible s < E, ties to the lower index, ascending, -1 padded."""
+    B, S, E = scores.shape
+    _need(q_pos, "q_pos", torch.int32, (B, S))
+    _need(scores, "scores", torch.float32)
+    if topk_idx is None:
+        topk_idx = torch.empty(B, S, k, dtype=torch.int32, device=scores.device)
+    _need(topk_idx, "topk_idx", torch.int32, (B, S, k))
+    if ws is None:
+        ws = workspace(_lib.CSA_WS_INDEXER_TOPK, B, S, E, k, scores.device)
+    check(_lib.load().csa_topk(B, S, ratio, k, q_pos.data_ptr(), scores.data_ptr(), E, topk_idx.data_ptr(),
+                               ws.data_ptr(), ws.numel(), _stream()), "csa_topk")
+    return topk_idx
+
+
 def _attn_common(q_pos, q, ring, cache, sink, out):
     B, S, H, d = q.shape
     _need(q_pos, "q_pos", torch.int32, (B, S))

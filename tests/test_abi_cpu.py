@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     names = declared_symbols()
     for want in ("csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode_fused",
                  "hca_decode_fused", "csa_workspace_size", "csa_get_device_status", "csa_state_reset",
-                 "csa_output_projection", "csa_q_projection", "csa_window_projection"):
+                 "csa_output_projection", "csa_q_projection", "csa_window_projection", "csa_indexer_scores",
+                 "csa_topk"):
         assert want in names
 
 
@@ -149,4 +150,10 @@ def test_host_side_argument_checks_launch_nothing(lib):
     assert lib.csa_window_projection(64, 7168, 512, 63, 1e4, 16, 16, 16, 16, 256, 256, null) == \
         _lib.CSA_ERR_UNSUPPORTED
     assert lib.csa_window_projection(64, 7168, 512, 64, 1e4, 16, 16, 16, 16, null, 0, null) == _lib.CSA_ERR_WORKSPACE
+    # the two halves of the indexer: scores required; selection needs scores and a 16-byte aligned row
+    assert lib.csa_indexer_scores(1, 1, 64, 128, 4, 16, 16, 16, 16, 128 * 8, 8, null, 256, 256, null) == \
+        _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_topk(1, 1, 4, 8, 16, null, 8, 16, 256, 4096, null) == _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_topk(1, 1, 4, 8, 16, 20, 8, 16, 256, 4096, null) == _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_topk(1, 1, 4, 4096, 16, 16, 8, 16, 256, 4096, null) == _lib.CSA_ERR_UNSUPPORTED
     assert lib.csa_last_error()

@@ -74,3 +74,76 @@ def test_two_gloo_ranks_shard_requests_and_reduce_time():
     line = res[0][6].strip().splitlines()
     assert len(line) == 1 and '"impl": "reference"' in line[0]
     assert res[1][6].strip() == ""
+
+
+def _tp_worker(rank: int, world: int, port: int, q) -> None:
+    """One rank of the tensor-parallel indexer over gloo, with the kernels replaced by the oracle."""
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank), MASTER_ADDR="127.0.0.1",
+                      MASTER_PORT=str(port))
+    try:
+        import types
+
+        import numpy as np
+        import torch.distributed as dist
+
+        import long_context_decode_c4a_b200.tp as tp
+        from oracle import csa_oracle as O
+        from synth import WORKLOADS, make_inputs
+
+        def fake_scores(q_pos, q_idx, w, idx_cache, ratio, scores=None):
+            B, S, H, _ = q_idx.shape
+            E = idx_cache.shape[1]
+            out = torch.zeros(B, S, E, dtype=torch.float64)
+            for b in range(B):
+                for i in range(S):
+                    vis = min((int(q_pos[b, i]) + 1) // ratio, E)
+                    out[b, i, :vis] = torch.from_numpy(O.indexer_scores(
+                        q_idx[b, i].double().numpy(), w[b, i].double().numpy(), idx_cache[b].double().numpy(), vis))
+            return out
+
+        def fake_topk(q_pos, scores, k, ratio):
+            B, S, E = scores.shape
+            out = torch.full((B, S, k), -1, dtype=torch.int32)
+            for b in range(B):
+                for i in range(S):
+                    vis = min((int(q_pos[b, i]) + 1) // ratio, E)
+                    sel = O.topk_select(scores[b, i, :vis].numpy(), k)
+                    out[b, i, :len(sel)] = torch.from_numpy(np.asarray(sel, dtype=np.int32))
+            return out
+
+        tp.ops = types.SimpleNamespace(indexer_scores=fake_scores, topk=fake_topk)
+        dist.init_process_group("gloo", rank=rank, world_size=world)
+        wl = WORKLOADS["pro_csa_decode_32k"].scaled(B=2, ctx=2048, topk=64)
+        inp = make_inputs(wl, seed=3)  # the same inputs on every rank
+        lo, hi = tp.head_shard(wl.H_I, rank, world)
+        sel = tp.tp_indexer_topk(inp["pos"], inp["q_idx"][:, :, lo:hi], inp["w"][:, :, lo:hi], inp["idx_cache"],
+                                 wl.topk)
+        full = fake_topk(inp["pos"], fake_scores(inp["pos"], inp["q_idx"], inp["w"], inp["idx_cache"], 4), wl.topk, 4)
+        dist.destroy_process_group()
+        q.put((rank, bool(torch.equal(sel, full)), (lo, hi)))
+    except Exception as e:  # noqa: BLE001
+        q.put((rank, "error", repr(e)))
+
+
+@pytest.mark.timeout(600)
+def test_tensor_parallel_indexer_over_two_gloo_ranks():
+    """[P1] "少读 KV 之前，Indexer 仍要给历史打分": each rank scores with half of the indexer heads, the
+    partial scores are summed by an all-reduce, and every rank selects the same entries as the
+    unsplit indexer."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_tp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        item = q.get(timeout=500)
+        res[item[0]] = item
+    for p in procs:
+        p.join(timeout=60)
+    assert res[0][1] != "error", res[0]
+    assert res[1][1] != "error", res[1]
+    assert res[0][1] is True and res[1][1] is True
+    assert res[0][2] == (0, 32) and res[1][2] == (32, 64)
