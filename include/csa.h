@@ -335,6 +335,18 @@ CSA_API int csa_output_projection(int M, int G, int Kg, int R, int D, const uint
                                   void* stream);
 
 /*
+ * csa_linear -- y = x . w^T on the tensor cores (the kernel of the projections around the layer),
+ * e.g. the compressor's streams ([P5] §2.1: each token's hidden state [hidden] -> the kv and score
+ * states [2*head_dim] of the main stream and [2*d_I] of the index stream).
+ *   x dev bf16 [M, K]; w dev bf16 [N, K]; y dev [M, N]: bf16 (y_is_f32 == 0, rounded from the fp32
+ *   accumulation) or float.
+ *   ws/ws_bytes: workspace of at least csa_workspace_size(CSA_WS_Q_PROJ, ...) (status word).
+ * Supported: N a multiple of 128, K a multiple of 64. Alignment: 16 bytes.
+ */
+CSA_API int csa_linear(int M, int N, int K, const uint16_t* x, const uint16_t* w, void* y, int y_is_f32, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/*
  * csa_q_projection -- the low-rank query path in front of the layer ([P1] section "低秩 Q：两次
  * 矩阵乘法接起来"), for M = B*S tokens:
  *   qa = x . wq_a^T                        (fp32, written to the caller's scratch qa)

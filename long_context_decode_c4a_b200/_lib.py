@@ -94,6 +94,7 @@ PROTOTYPES = {
                                    c_int64, c_int, c_void_p, c_void_p, c_size_t, c_void_p]),
     "csa_topk": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_size_t,
                          c_void_p]),
+    "csa_linear": (c_int, [c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
     "csa_q_projection": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_float, c_float, c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                  c_void_p]),

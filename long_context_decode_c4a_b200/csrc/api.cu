@@ -647,6 +647,29 @@ int csa_output_projection(int M, int G, int Kg, int R, int D, const uint16_t* o,
                   (uint64_t)G * R, P2, 1, dev->sms, st);
 }
 
+int csa_linear(int M, int N, int K, const uint16_t* x, const uint16_t* w, void* y, int y_is_f32, void* ws,
+               size_t ws_bytes, void* stream) {
+  CSA_CHECK_ARG(M > 0 && N > 0 && K > 0, "sizes must be positive");
+  CSA_CHECK_ARG(x && w && y, "null pointer");
+  CSA_CHECK_ARG(aligned(x, 16) && aligned(w, 16) && aligned(y, 16), "pointers must be 16-byte aligned");
+  CSA_CHECK_SUP(N % 128 == 0 && K % 64 == 0, "N must be a multiple of 128 and K of 64");
+  if (int rc = check_ws(ws, ws_bytes, kStatusBytes)) return rc;
+  DeviceInfo* dev;
+  if (int rc = device_info(&dev)) return rc;
+  GemmParams P{};
+  P.M = M;
+  P.N = N;
+  P.K = K;
+  // fp32 output may be split over K (fp32 reductions); bf16 output is stored by one CTA per tile.
+  P.splits = y_is_f32 ? gemm_splits((long long)(N / 128) * ((M + 127) / 128), K / 64, dev->sms) : 1;
+  P.ldc = N;
+  P.c = y;
+  P.c_mode = !y_is_f32 ? kGemmOutBf16 : (P.splits > 1 ? kGemmOutF32Add : kGemmOutF32);
+  P.status = reinterpret_cast<uint32_t*>(ws);
+  return run_gemm(x, (uint64_t)K, (uint64_t)M, (uint64_t)K, w, (uint64_t)K, (uint64_t)N, (uint64_t)K, P, 1, dev->sms,
+                  static_cast<cudaStream_t>(stream));
+}
+
 int csa_q_projection(int M, int hidden, int q_rank, int H, int d, int rope_dim, float rope_base, float eps,
                      const int32_t* pos, const uint16_t* x, const uint16_t* wq_a, const uint16_t* gamma,
                      const uint16_t* wq_b, float* qa, uint16_t* qr, uint16_t* q, void* ws, size_t ws_bytes,

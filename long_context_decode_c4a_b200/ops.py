@@ -420,6 +420,31 @@ def output_projection(o: torch.Tensor, wo_a: torch.Tensor, wo_b: torch.Tensor, r
     return r, y
 
 
+def linear(x: torch.Tensor, w: torch.Tensor, out_dtype: torch.dtype = torch.bfloat16, y: Optional[torch.Tensor] = None,
+           ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = x . w^T for x [M, K], w [N, K] bf16; y bf16 or fp32 [M, N]."""
+    M, K = x.shape
+    N = w.shape[0]
+    _need(x, "x", torch.bfloat16)
+    _need(w, "w", torch.bfloat16, (N, K))
+    if y is None:
+        y = torch.empty(M, N, dtype=out_dtype, device=x.device)
+    _need(y, "y", out_dtype, (M, N))
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("out_dtype must be bf16 or fp32")
+    if ws is None:
+        ws = workspace(_lib.CSA_WS_Q_PROJ, 1, 1, 1, 1, x.device)
+    check(_lib.load().csa_linear(M, N, K, x.data_ptr(), w.data_ptr(), y.data_ptr(), int(out_dtype == torch.float32),
+                                 ws.data_ptr(), ws.numel(), _stream()), "csa_linear")
+    return y
+
+
+def compressor_streams(x: torch.Tensor, w_kv: torch.Tensor, w_score: torch.Tensor):
+    """The compressor's per-token states from the hidden states x [M, hidden]: kv = x . w_kv^T and
+    score = x . w_score^T (bf16 [M, width]), the inputs of csa_compress."""
+    return linear(x, w_kv), linear(x, w_score)
+
+
 def q_projection(x: torch.Tensor, wq_a: torch.Tensor, gamma: torch.Tensor, wq_b: torch.Tensor, pos: torch.Tensor,
                  H: int = 128, d: int = 512, rope_dim: int = 64, rope_base: float = 10000.0, eps: float = 1e-6,
                  q: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):

@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
     for want in ("csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_attn", "csa_decode_fused",
                  "hca_decode_fused", "csa_workspace_size", "csa_get_device_status", "csa_state_reset",
                  "csa_output_projection", "csa_q_projection", "csa_window_projection", "csa_indexer_scores",
-                 "csa_topk"):
+                 "csa_topk", "csa_linear"):
         assert want in names
 
 
@@ -156,4 +156,6 @@ def test_host_side_argument_checks_launch_nothing(lib):
     assert lib.csa_topk(1, 1, 4, 8, 16, null, 8, 16, 256, 4096, null) == _lib.CSA_ERR_INVALID_ARG
     assert lib.csa_topk(1, 1, 4, 8, 16, 20, 8, 16, 256, 4096, null) == _lib.CSA_ERR_INVALID_ARG
     assert lib.csa_topk(1, 1, 4, 4096, 16, 16, 8, 16, 256, 4096, null) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_linear(64, 1000, 7168, 16, 16, 16, 0, 256, 256, null) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_linear(64, 1024, 7168, null, 16, 16, 0, 256, 256, null) == _lib.CSA_ERR_INVALID_ARG
     assert lib.csa_last_error()

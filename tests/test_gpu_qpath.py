@@ -104,3 +104,22 @@ def test_window_projection(ops, M, hidden):
     x, wkv, pos = np64(inp["x"]), np64(inp["wkv"]), np64(inp["pos"])
     ref = O.window_projection(x, wkv, pos)
     _rel_close(np64(win), ref, 2.0 ** -6, 1e-2 * _rms(ref), "window rows")
+
+
+@pytest.mark.parametrize("M,N", [(64, 1024), (64, 256), (130, 1024)])
+def test_compressor_stream_projection(ops, M, N):
+    """The compressor's kv and score states from the hidden states ([P5] §2.1: [hidden] -> [2 head_dim]
+    for the main stream, [2 d_I] for the index stream), rounded to bf16, and the fp32 variant."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(M + N)
+    x = torch.randn(M, 7168, generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn(N, 7168, generator=g, device="cuda") / 84.7).to(torch.bfloat16)
+    kv, score = ops.compressor_streams(x, w, w)
+    y32 = ops.linear(x, w, torch.float32)
+    torch.cuda.synchronize()
+    exact = np64(x) @ np64(w).T
+    scale = _rms(exact)
+    assert np.max(np.abs(np64(y32) - exact)) <= 1e-4 * scale, "fp32 linear"
+    # bf16: one bf16 step (kernel and oracle both rounded) plus the accumulation error
+    _bf16_close(np64(kv), O.bf16(exact), scale, "kv stream")
+    assert torch.equal(kv, score)
