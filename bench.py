@@ -156,6 +156,12 @@ def max_over_ranks(x: float, world: int) -> float:
 
 # ------------------------------------------------------------------------------ per-step byte / flop ledgers
 
+def graph_rounds(requested: int, steps: int, sets: int) -> int:
+    """Rounds of the input-set sequence per CUDA graph: as many as requested, but no more than the
+    timed steps hold, so that a graph always serves when there are at least `sets` steps."""
+    return max(1, min(requested, steps // max(1, sets)))
+
+
 def decode_bytes(wl):
     """Algorithmic HBM bytes per query of each kernel of one CSA/HCA decode step."""
     E = wl.max_entries
@@ -221,9 +227,12 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
     for i in range(args.warmup):
         call(i)
     torch.cuda.synchronize()
-    # One CUDA graph holds one step of every input set (the launches keep their programmatic
-    # dependencies); the timed region replays it and launches any remaining steps directly.
+    # One CUDA graph holds `reps` rounds of one step of every input set (the launches keep their
+    # programmatic dependencies, which a graph boundary ends); the timed region replays it and
+    # launches any remaining steps directly.
     graph = None
+    reps = graph_rounds(getattr(args, "graph_reps", 1), args.steps, len(preps))
+    per_graph = reps * len(preps)
     if args.graph:
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
@@ -234,10 +243,10 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            for i in range(len(preps)):
-                call(i)
+            for i in range(per_graph):
+                call(i % len(preps))
         torch.cuda.synchronize()
-        for _ in range(max(1, args.warmup // len(preps))):
+        for _ in range(max(1, args.warmup // per_graph)):
             graph.replay()
         torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -248,10 +257,10 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
     t0.record()
     k = 0
     if graph is not None:
-        while k + len(preps) <= args.steps:
+        while k + per_graph <= args.steps:
             graph.replay()
-            k += len(preps)
-            if (k // len(preps)) % 4 == 0:
+            k += per_graph
+            if (k // per_graph) % max(1, 4 // reps) == 0:
                 clocks.sample()
     for kk in range(k, args.steps):
         call(kk)
@@ -590,6 +599,9 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=0, help="requests per GPU (default: the workload's)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the short runs of the other configurations")
+    ap.add_argument("--graph-reps", type=int, default=10,
+                    help="rounds of the input-set sequence captured in one CUDA graph (a graph boundary "
+                         "ends the programmatic overlap of consecutive launches)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="launch every timed step from the host instead of replaying a CUDA graph")
     args = ap.parse_args(argv)

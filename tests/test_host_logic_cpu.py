@@ -74,3 +74,16 @@ def test_decode_bytes_ledger():
     E = wl.max_entries
     assert per_q["indexer"] == E * wl.d_I * 2 + wl.H_I * wl.d_I * 2 + wl.H_I * 4 + E * 4
     assert math.isclose(per_q["attention"] / 1e6, 1.44, rel_tol=0.01)
+
+
+def test_graph_rounds_fit_the_timed_steps():
+    """The CUDA graph of the timed loop holds whole rounds of the input-set sequence and never more
+    steps than the run times (the rest are launched directly)."""
+    assert bench.graph_rounds(10, 200, 4) == 10
+    assert bench.graph_rounds(10, 12, 4) == 3
+    assert bench.graph_rounds(10, 3, 4) == 1
+    assert bench.graph_rounds(1, 200, 4) == 1
+    assert bench.graph_rounds(10, 20, 2) == 10
+    for steps in range(1, 60):
+        r = bench.graph_rounds(10, steps, 4)
+        assert r >= 1 and (r * 4 <= steps or steps < 4)
