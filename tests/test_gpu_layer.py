@@ -55,7 +55,7 @@ def check_csa_request(wl, inp_np, st, out, cache32, b):
     assert np.max(np.abs(gi - ref["idx_entry"])) <= 5e-3 + np.max(np.abs(ref["idx_entry"])) * 2 ** -8
     sel = check_topk(np64(st.topk_idx[b]), ref["scores"], wl.topk, f"b={b}")
     if not np.array_equal(np.sort(sel), ref["topk"][: len(sel)]):
-        # Near-tie swap: judge the attention on the GPU's own selection.
+        # Near-tie swap: check the attention on the GPU's own selection.
         ref_out = O.attend_query(inp_np["q"][b, 0], t, wl.W, ref["ring"], wl.W, ref["cache"], sel.tolist(),
                                  inp_np["sink"], 1 / math.sqrt(wl.d), wl.rope_dim, wl.rope_base)
     else:
