@@ -1,0 +1,130 @@
+"""Mutation check of the oracle's pins.
+
+Each case plants one plausible mistake (a dropped term, a wrong sign, index, axis or operand) in a
+copy of the oracle built in memory from its source text, on the CPU; the oracle's file is never
+written. The pins of test_oracle_pins.py then run against the mutant, and at least one of them must
+fail. A control case runs the same pins against the unmodified source, which must pass them all, so a
+broken runner cannot pass for a caught mutant.
+
+Not listed, because no test can tell it apart from the oracle: dropping the +0.0 that folds -0
+into +0 before the top-k sort (numpy's sort already orders -0 and +0 as equal)."""
+
+import itertools
+import os
+import types
+
+import numpy as np
+import pytest
+
+from tests import test_oracle_pins as pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ORACLE_SRC = os.path.join(ROOT, "oracle", "csa_oracle.py")
+
+# name -> (text in the oracle, the mistake put in its place)
+MUTATIONS = {
+    # compressor
+    "state_machine_wrong_halves": (
+        "slot_kv = np.concatenate([state_kv[:r, :d], state_kv[r:, d:]], axis=0)",
+        "slot_kv = np.concatenate([state_kv[:r, d:], state_kv[r:, :d]], axis=0)"),
+    "direct_formula_wrong_half": (
+        "slot_kv = np.concatenate([kv[prev, :d], kv[cur, d:]], axis=0)",
+        "slot_kv = np.concatenate([kv[prev, d:], kv[cur, d:]], axis=0)"),
+    "state_not_rolled": ("        state_kv[:r] = state_kv[r:]\n", "        pass\n"),
+    "softmax_over_channels": ("wts = e / np.sum(e, axis=0)", "wts = e / np.sum(e, axis=1, keepdims=True)"),
+    "entry_position_off_by_one": ("rope(rms_norm(pooled, gamma, eps), g * ratio,",
+                                  "rope(rms_norm(pooled, gamma, eps), g * ratio + 1,"),
+    "rmsnorm_without_eps": ("/ np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)",
+                            "/ np.sqrt(np.mean(x * x, axis=-1, keepdims=True))"),
+    "entry_visible_one_early": ("return (t + 1) // ratio", "return t // ratio + 1"),
+    # RoPE
+    "rope_wrong_sign": ("y[..., head + 1::2] = even * s + odd * c", "y[..., head + 1::2] = -even * s + odd * c"),
+    # indexer and top-k
+    "indexer_without_relu": ("return np.maximum(logits, 0.0) @", "return logits @"),
+    "indexer_relu_after_weighting": (
+        "return np.maximum(logits, 0.0) @ np.asarray(w, dtype=np.float64)",
+        "return np.maximum(logits @ np.asarray(w, dtype=np.float64), 0.0)"),
+    "ties_to_higher_index": ("order = np.lexsort((np.arange(n), -key, nan_last))",
+                             "order = np.lexsort((-np.arange(n), -key, nan_last))"),
+    "selection_in_score_order": ("sel = np.sort(order[: min(k, n)])", "sel = order[: min(k, n)]"),
+    # attention
+    "window_shifted": ("return list(range(max(0, t - W + 1), t + 1))", "return list(range(max(0, t - W), t))"),
+    "sink_left_out_of_the_max": ("m = np.maximum(np.max(logits, axis=1), sink)", "m = np.max(logits, axis=1)"),
+    "sink_not_in_denominator": ("denom = np.sum(e, axis=1) + np.exp(sink - m)", "denom = np.sum(e, axis=1)"),
+    "logits_unscaled": ("logits = scale * (q @ cand.T)", "logits = (q @ cand.T)"),
+    "output_rotated_forward": ("return rope(o, t, rope_dim, rope_base, inverse=True)",
+                               "return rope(o, t, rope_dim, rope_base)"),
+    # output projection
+    "projection_wrong_group_weights": ('r = np.einsum("mgk,grk->mgr", og, wo_a)',
+                                       'r = np.einsum("mgk,grk->mgr", og, wo_a[::-1])'),
+    "projection_r_not_rounded": ("y = rb.reshape(M, G * R) @ wo_b.T", "y = r.reshape(M, G * R) @ wo_b.T"),
+    # query path and window rows
+    "q_without_gamma": ("qr = bf16(rms_norm(qa, gamma, eps))", "qr = bf16(rms_norm(qa, 1.0, eps))"),
+    "q_norm_over_all_heads": ("q = qraw / np.sqrt(np.mean(qraw * qraw, axis=-1, keepdims=True) + eps)",
+                              "q = qraw / np.sqrt(np.mean(qraw * qraw, axis=(-2, -1), keepdims=True) + eps)"),
+    "q_rotated_at_next_position": ("q[m] = rope(q[m], float(pos[m]), rope_dim, rope_base)",
+                                   "q[m] = rope(q[m], float(pos[m]) + 1.0, rope_dim, rope_base)"),
+    "window_row_not_rotated": (
+        "return np.stack([rope(w[m], float(pos[m]), rope_dim, rope_base) for m in range(x.shape[0])])",
+        "return w.copy()"),
+}
+
+
+def _oracle_from(source: str) -> types.ModuleType:
+    mod = types.ModuleType("csa_oracle_mutant")
+    mod.__file__ = ORACLE_SRC
+    exec(compile(source, ORACLE_SRC, "exec"), mod.__dict__)
+    return mod
+
+
+def _pin_calls(golden_dir):
+    """Every pin of test_oracle_pins.py with each of its parameter sets, in file order."""
+    calls = []
+    for name, fn in vars(pins).items():
+        if not (name.startswith("test_") and callable(fn)):
+            continue
+        axes = []
+        for mark in getattr(fn, "pytestmark", []):
+            if mark.name != "parametrize":
+                continue
+            argnames, values = mark.args[0], mark.args[1]
+            argnames = [a.strip() for a in argnames.split(",")] if isinstance(argnames, str) else list(argnames)
+            axes.append([dict(zip(argnames, v if len(argnames) > 1 else (v,))) for v in values])
+        for combo in itertools.product(*axes) if axes else [()]:
+            kwargs = {}
+            for part in combo:
+                kwargs.update(part)
+            if "golden_dir" in fn.__code__.co_varnames[:fn.__code__.co_argcount]:
+                kwargs["golden_dir"] = golden_dir
+            calls.append((name, fn, kwargs))
+    return calls
+
+
+def _first_failing_pin(monkeypatch, module, golden_dir):
+    monkeypatch.setattr(pins, "O", module)
+    for name, fn, kwargs in _pin_calls(golden_dir):
+        try:
+            with np.errstate(all="ignore"):
+                fn(**kwargs)
+        except Exception as exc:          # an assertion, or the mutant breaking a shape
+            return f"{name}{kwargs or ''}: {type(exc).__name__}"
+    return None
+
+
+def _source():
+    with open(ORACLE_SRC) as f:
+        return f.read()
+
+
+def test_control_unmodified_oracle_passes_every_pin(monkeypatch, golden_dir):
+    assert len(_pin_calls(golden_dir)) >= 30
+    assert _first_failing_pin(monkeypatch, _oracle_from(_source()), golden_dir) is None
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_fails_a_pin(monkeypatch, golden_dir, name):
+    before, after = MUTATIONS[name]
+    src = _source()
+    assert src.count(before) == 1, f"{name}: the text to mutate must occur exactly once"
+    caught = _first_failing_pin(monkeypatch, _oracle_from(src.replace(before, after)), golden_dir)
+    assert caught is not None, f"{name}: no pin fails"

@@ -33,7 +33,8 @@ def test_bf16_rounding_matches_known_values():
     assert O.bf16(np.inf) == np.inf and np.isnan(O.bf16(np.nan))
     # Every bf16 value round-trips.
     bits = np.arange(0, 1 << 16, 7, dtype=np.uint32) << 16
-    vals = bits.view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):          # the NaN patterns among the bits
+        vals = bits.view(np.float32).astype(np.float64)
     fin = np.isfinite(vals)
     assert np.array_equal(O.bf16(vals[fin]), vals[fin])
 
@@ -369,6 +370,11 @@ def test_large_sink_stays_finite():
     q = np.ones((1, 4)); c = np.ones((3, 4)) * 0.1
     o = O.mqa_with_sink(q, c, np.array([1000.0]), 1.0)
     assert np.all(np.isfinite(o)) and np.max(np.abs(o)) < 1e-300
+    # A sink 720 above the three equal logits (0.4): exp(720) overflows float64, but with the sink in
+    # the max every exponent is <= 0 and the output keeps its closed form 0.1 * 3 e^-720 / (1 + 3 e^-720)
+    # = 0.3 e^-720 (a subnormal, about 2e-314), which an overflowed denominator would flush to 0.
+    o = O.mqa_with_sink(q, c, np.array([720.4]), 1.0)
+    assert np.allclose(o, 0.3 * math.exp(-720.0), rtol=1e-6, atol=0.0) and np.all(o > 0)
 
 
 def test_rmsnorm_eps_matters_for_small_vectors():
@@ -426,6 +432,19 @@ def test_output_projection_groups_are_independent_and_linear():
     for g in range(G):
         assert np.allclose(r[:, g * R:(g + 1) * R], o[:, g * Kg:(g + 1) * Kg] @ wa[g].T, rtol=1e-14, atol=1e-12)
     assert np.array_equal(rb, O.bf16(r))
+
+
+def test_output_projection_rounds_r_before_the_second_product():
+    """R20 on values fixed by hand: o = [1, 2^-9] summed by Wo_a = [1, 1] gives r = 1 + 2^-9, which
+    lies below half a bf16 step above 1, so the rounded r is 1 and y = 1 * 3 = 3 exactly; o = [1,
+    3 * 2^-8] gives r = 1 + 3 * 2^-8, half-way between two bf16 values, which rounds to the even
+    one, 1 + 2^-6, and y = 3 + 3 * 2^-6."""
+    wa = np.ones((1, 1, 2))
+    wb = np.array([[3.0]])
+    for second, r_exact, y_exact in ((2.0 ** -9, 1.0 + 2.0 ** -9, 3.0),
+                                     (3 * 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, 3.0 + 3 * 2.0 ** -6)):
+        r, rb, y = O.output_projection(np.array([[1.0, second]]), wa, wb)
+        assert r[0, 0] == r_exact and y[0, 0] == y_exact
 
 
 # ----------------------------------------------------------------------------- query path
