@@ -364,6 +364,26 @@ def test_reads_per_query_edge_cases():
     assert O.reads_per_query(1048575, 128, 4, 1024) == 1152
 
 
+def test_prefill_totals_match_arithmetic_series():
+    """An 8192-token CSA prefill from an empty cache, totalled over its queries and checked against
+    sums of arithmetic series rather than a loop. u = t + 1 runs over 1..8192.
+
+    Visible entries: floor(u/4) is k for the four values u = 4k..4k+3, and 2048 at u = 8192. The
+    sum is 4 (1 + ... + 2047) + 2048 = 8,386,560 (query, entry) pairs for the indexer.
+
+    Reads: the window part min(128, u) sums to 128 * 129 / 2 + (8192 - 128) * 128 = 1,040,448. The
+    selected part min(1024, floor(u/4)) sums to 4 (1 + ... + 1023) over u < 4096, plus 1024 for each
+    of the 4097 values u >= 4096, which is 6,290,432. The total is 7,330,880 reads."""
+    S = 8192
+    assert sum(O.visible_entries(t, 4) for t in range(S)) == 4 * (2047 * 2048 // 2) + 2048 == 8_386_560
+    window = 128 * 129 // 2 + (S - 128) * 128
+    selected = 4 * (1023 * 1024 // 2) + 4097 * 1024
+    assert (window, selected) == (1_040_448, 6_290_432)
+    assert sum(O.reads_per_query(t, 128, 4, 1024) for t in range(S)) == window + selected == 7_330_880
+    # HCA (ratio 128, every visible entry): floor(u/128) sums to 128 (1 + ... + 63) + 64.
+    assert sum(O.reads_per_query(t, 128, 128, None) for t in range(S)) == window + 128 * (63 * 64 // 2) + 64
+
+
 def test_large_sink_stays_finite():
     """R6: the running max includes the sink, so a sink far above every logit gives an
     output near zero instead of overflowing."""
