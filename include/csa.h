@@ -19,6 +19,9 @@
  *     out-of-range index, records a code in the workspace status word and returns.
  *     csa_get_device_status reads it.
  *   - Positions t are absolute token positions (0-based). Batch strides are in elements.
+ *   - Every size that counts work (B, S, M, the widths) must be at least 1: a call with no work
+ *     (B = 0, S = 0, M = 0) is refused with CSA_ERR_INVALID_ARG and enqueues nothing, so a
+ *     caller with an empty batch skips the call.
  *   - Thread safety: the library keeps no state except a thread-local error string.
  */
 #ifndef CSA_H_

@@ -159,3 +159,41 @@ def test_host_side_argument_checks_launch_nothing(lib):
     assert lib.csa_linear(64, 1000, 7168, 16, 16, 16, 0, 256, 256, null) == _lib.CSA_ERR_UNSUPPORTED
     assert lib.csa_linear(64, 1024, 7168, null, 16, 16, 0, 256, 256, null) == _lib.CSA_ERR_INVALID_ARG
     assert lib.csa_last_error()
+
+
+def test_calls_with_no_work_are_refused_before_any_launch(lib):
+    """B = 0, S = 0 or M = 0: every entry returns CSA_ERR_INVALID_ARG from its host-side checks (on a
+    machine without a GPU, so no CUDA call was reached) and names the size in its error text."""
+    cfg = _lib.CompressorCfg(4, 1, 512, 64, 10000.0, 1e-6)
+    null, ws = None, 1 << 20
+    calls = {
+        "compress S=0": lambda: lib.csa_compress(ctypes.byref(cfg), 1, 0, 16, 16, 16, 16, 16, 16, 16, 4096 * 512, 4096,
+                                                 null, null),
+        "compress B=0": lambda: lib.csa_compress(ctypes.byref(cfg), 0, 4, 16, 16, 16, 16, 16, 16, 16, 4096 * 512, 4096,
+                                                 null, null),
+        "indexer_topk S=0": lambda: lib.csa_indexer_topk(1, 0, 64, 128, 4, 8, 16, 16, 16, 16, 128 * 8, 8, 16, null,
+                                                         256, ws, null),
+        "indexer_topk B=0": lambda: lib.csa_indexer_topk(0, 1, 64, 128, 4, 8, 16, 16, 16, 16, 128 * 8, 8, 16, null,
+                                                         256, ws, null),
+        "indexer_scores S=0": lambda: lib.csa_indexer_scores(1, 0, 64, 128, 4, 16, 16, 16, 16, 128 * 8, 8, 16, 256,
+                                                             ws, null),
+        "topk S=0": lambda: lib.csa_topk(1, 0, 4, 8, 16, 16, 8, 16, 256, ws, null),
+        "sparse_attn S=0": lambda: lib.csa_sparse_attn(1, 0, 128, 512, 64, 1e4, 0.05, 16, 16, 16, 512 * 128, 128, 128,
+                                                       16, 512 * 8, 8, 16, 8, 16, 16, 0, 256, ws, null),
+        "hca_attn S=0": lambda: lib.hca_attn(1, 0, 128, 512, 64, 1e4, 0.05, 128, 16, 16, 16, 512 * 128, 128, 128, 16,
+                                             512 * 8, 8, 16, 16, 0, 256, ws, null),
+        "output_projection M=0": lambda: lib.csa_output_projection(0, 16, 4096, 1024, 7168, 16, 16, 16, 16, 16, 256,
+                                                                   ws, null),
+        "q_projection M=0": lambda: lib.csa_q_projection(0, 7168, 1536, 128, 512, 64, 1e4, 1e-6, 16, 16, 16, 16, 16,
+                                                         16, 16, 16, 256, ws, null),
+        "window_projection M=0": lambda: lib.csa_window_projection(0, 7168, 512, 64, 1e4, 16, 16, 16, 16, 256, ws,
+                                                                   null),
+        "linear M=0": lambda: lib.csa_linear(0, 1024, 7168, 16, 16, 16, 0, 256, ws, null),
+    }
+    for name, call in calls.items():
+        assert call() == _lib.CSA_ERR_INVALID_ARG, name
+        assert b"positive" in lib.csa_last_error(), name
+    n = ctypes.c_size_t()
+    for kind in (_lib.CSA_WS_INDEXER_TOPK, _lib.CSA_WS_SPARSE_ATTN, _lib.CSA_WS_HCA_ATTN):
+        assert lib.csa_workspace_size(kind, 1, 0, 256, 8, ctypes.byref(n)) == _lib.CSA_ERR_INVALID_ARG
+
