@@ -67,6 +67,22 @@ MUTATIONS = {
     "window_row_not_rotated": (
         "return np.stack([rope(w[m], float(pos[m]), rope_dim, rope_base) for m in range(x.shape[0])])",
         "return w.copy()"),
+    # order of the modules in one decode step
+    "indexer_scored_before_the_in_step_index_entry": (
+        'scores = indexer_scores(inp["q_idx"][b, 0], inp["w"][b, 0], icache, vis)',
+        'scores = indexer_scores(inp["q_idx"][b, 0], inp["w"][b, 0], inp["idx_cache"][b], vis)'),
+    "ring_written_after_attention": (
+        'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, cache, sel,',
+        'out = attend_query(inp["q"][b, 0], t, W, inp["ring"][b], ring_cap, cache, sel,'),
+    "entry_written_after_attention": (
+        'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, cache, sel,',
+        'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, inp["cache"][b], sel,'),
+    "hca_ring_written_after_attention": (
+        'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, cache, list(range(vis)),',
+        'out = attend_query(inp["q"][b, 0], t, W, inp["ring"][b], ring_cap, cache, list(range(vis)),'),
+    "hca_entry_written_after_attention": (
+        'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, cache, list(range(vis)),',
+        'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, inp["cache"][b], list(range(vis)),'),
 }
 
 

@@ -520,3 +520,108 @@ def test_window_projection_one_hot_closed_form():
     w = O.window_projection(x, wkv, pos)
     for m in range(M):
         assert np.allclose(w[m], _complex_rotate(x[m, sel], pos[m], 64, 10000.0), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- decode step composition
+
+def _prefill_inputs(rng, S, H, d, ratio):
+    """Random float64 inputs of one request's prefill segment from position 0 (tiny shapes)."""
+    ov = ratio == 4
+    width = 2 * d if ov else d
+    inp = dict(kv=rng.standard_normal((1, S, width)), score=rng.standard_normal((1, S, width)),
+               win_kv=rng.standard_normal((1, S, d)), q=rng.standard_normal((1, S, H, d)) / math.sqrt(d) * 3,
+               sink=rng.standard_normal(H), gamma=np.ones(d), pos=np.arange(S)[None, :])
+    if ov:
+        inp.update(idx_kv=rng.standard_normal((1, S, 256)), idx_score=rng.standard_normal((1, S, 256)),
+                   q_idx=rng.standard_normal((1, S, 4, 128)), w=rng.standard_normal((1, S, 4)),
+                   idx_gamma=np.ones(128))
+    return inp
+
+
+def _decode_inputs_at(pre, t, W, ratio, rng):
+    """The decode-step inputs of token t, built from a prefill segment the way a serving loop holds
+    them before the step: the compressor states after tokens 0..t-1 (token-by-token machine), the
+    cache rows of every group completed before t, a W-slot ring with the window rows of tokens
+    t-W+1..t-1 at slot p % W, and token t's own streams. Cache rows not yet written and the ring slot
+    token t will take hold stale values (random draws), as pooled memory does."""
+    d = pre["win_kv"].shape[2]
+    E = pre["win_kv"].shape[1] // ratio
+    main = O.CompressorCfg(ratio, d)
+    skv, ssc = O.init_state(main)
+    done = O.compress_tokens(main, skv, ssc, 0, pre["kv"][0, :t], pre["score"][0, :t], pre["gamma"])
+    cache = O.bf16(rng.standard_normal((E, d)))
+    for g, e in done.items():
+        cache[g] = O.bf16(e)
+    ring = O.bf16(rng.standard_normal((W, d)))
+    for p in range(max(0, t - W + 1), t):
+        ring[p % W] = pre["win_kv"][0, p]
+    one = lambda x: x[:, t:t + 1]
+    inp = dict(state_kv=skv[None], state_score=ssc[None], cache=cache[None], ring=ring[None],
+               kv=one(pre["kv"]), score=one(pre["score"]), win_kv=one(pre["win_kv"]), q=one(pre["q"]),
+               sink=pre["sink"], gamma=pre["gamma"], pos=np.array([[t]]))
+    if "idx_kv" in pre:
+        idx = O.CompressorCfg(ratio, 128)
+        ikv, isc = O.init_state(idx)
+        idone = O.compress_tokens(idx, ikv, isc, 0, pre["idx_kv"][0, :t], pre["idx_score"][0, :t],
+                                  pre["idx_gamma"])
+        icache = O.bf16(rng.standard_normal((E, 128)))
+        for g, e in idone.items():
+            icache[g] = O.bf16(e)
+        inp.update(idx_state_kv=ikv[None], idx_state_score=isc[None], idx_cache=icache[None],
+                   idx_kv=one(pre["idx_kv"]), idx_score=one(pre["idx_score"]), q_idx=one(pre["q_idx"]),
+                   w=one(pre["w"]), idx_gamma=pre["idx_gamma"])
+    return inp
+
+
+@pytest.mark.parametrize("t", [3, 11, 13, 31, 63, 70, 127])
+def test_csa_decode_step_equals_prefill_query_at_the_same_position(t):
+    """The decode step composes its modules in the pages' order ([P5] §2: compressor, then the index
+    module over the index cache, then attention over window + selected entries): the compressor step
+    of token t, which completes entry t // 4 when (t + 1) % 4 == 0, lands in both caches before the
+    indexer scores and attention reads them, and token t's window row is in the ring before attention.
+    A decode step fed the state a serving loop holds after tokens 0..t-1 must therefore reproduce the
+    prefill's query t ([P1] "压缩条目必须等整组完成后才可见": every query sees (t + 1) // 4 entries),
+    whose parallel compression is pinned against the state machine above. t covers group completion
+    and non-completion, all-visible selection (t < 32 with top-k 8) and t below and above the window."""
+    S, H, d, W, topk = 128, 8, 512, 16, 8
+    rng = np.random.default_rng(20)
+    pre = _prefill_inputs(rng, S, H, d, 4)
+    dec_in = _decode_inputs_at(pre, t, W, 4, np.random.default_rng(21))
+    dec = O.csa_decode_request(dec_in, 0, H=H, d=d, W=W, topk=topk)
+    ref = O.csa_prefill(pre, 0, [t], H=H, d=d, W=W, topk=topk)
+    q = ref["queries"][t]
+    vis = (t + 1) // 4
+    assert dec["scores"].shape == (vis,)
+    assert np.allclose(dec["scores"], q["scores"], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(dec["topk"], q["topk"])
+    assert np.allclose(dec["out"], q["out"], rtol=1e-10, atol=1e-12)
+    if (t + 1) % 4 == 0:
+        g = t // 4
+        assert np.allclose(dec["entry"], ref["entries"][g], rtol=1e-12, atol=1e-12)
+        assert np.allclose(dec["idx_entry"], ref["idx_entries"][g], rtol=1e-12, atol=1e-12)
+        assert np.array_equal(dec["cache"][g], ref["cache"][g])
+        assert np.array_equal(dec["idx_cache"][g], ref["idx_cache"][g])
+    else:
+        assert dec["entry"] is None and dec["idx_entry"] is None
+    assert np.array_equal(dec["ring"][t % W], pre["win_kv"][0, t])
+
+
+@pytest.mark.parametrize("t", [127, 255, 300, 383])
+def test_hca_decode_step_equals_prefill_query_at_the_same_position(t):
+    """HCA ([P5] §3: C128A, no index module): the C128A step of token t completes entry t // 128 when
+    (t + 1) % 128 == 0 and is in the cache before attention reads every visible entry; token t's
+    window row is in the ring first. The decode step must reproduce the HCA prefill's query t."""
+    S, H, d, W, ratio = 384, 4, 512, 16, 128
+    rng = np.random.default_rng(22)
+    pre = _prefill_inputs(rng, S, H, d, ratio)
+    dec_in = _decode_inputs_at(pre, t, W, ratio, np.random.default_rng(23))
+    dec = O.hca_decode_request(dec_in, 0, H=H, d=d, W=W, ratio=ratio)
+    ref = O.csa_prefill(pre, 0, [t], H=H, d=d, W=W, topk=0, ratio=ratio, with_indexer=False)
+    assert np.allclose(dec["out"], ref["queries"][t]["out"], rtol=1e-10, atol=1e-12)
+    if (t + 1) % ratio == 0:
+        g = t // ratio
+        assert np.allclose(dec["entry"], ref["entries"][g], rtol=1e-12, atol=1e-12)
+        assert np.array_equal(dec["cache"][g], ref["cache"][g])
+    else:
+        assert dec["entry"] is None
+    assert np.array_equal(dec["ring"][t % W], pre["win_kv"][0, t])
