@@ -308,7 +308,8 @@ CSA_API int csa_topk(int B, int S, int ratio, int topk, const int32_t* q_pos, co
  * memory; every GPU that loads the library holds it until the process exits. Arguments and
  * results are those of csa_indexer_topk, without scores_opt and ws.
  * Limits: max_entries <= 16384 and B*S*max_entries <= 1,048,576; larger calls return
- * CSA_ERR_UNSUPPORTED without launching.
+ * CSA_ERR_UNSUPPORTED without launching. Every argument is checked as csa_indexer_topk checks it
+ * before the array is touched, so a refused call writes nothing to the device.
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress), so
  * make that first call before any stream capture on that device. Every call shares the array:
  * calls that overlap on the GPU (unordered streams) race. Device-side status (timeouts, bounds) is

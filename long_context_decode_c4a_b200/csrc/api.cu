@@ -487,6 +487,15 @@ int run_gemm(const void* A, uint64_t a_cols, uint64_t a_rows, uint64_t lda, cons
 }
 
 }  // namespace
+
+int check_indexer_topk_args(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
+                            const uint16_t* q_idx, const float* w, const uint16_t* idx_cache, int64_t idx_bstride,
+                            int max_entries, const int32_t* topk_idx) {
+  IndexerArgs a{B, S, H_I, d_I, ratio, topk, q_pos, q_idx, w, idx_cache, idx_bstride, max_entries,
+                const_cast<int32_t*>(topk_idx), nullptr, nullptr, 0};
+  return check_indexer_args(a);
+}
+
 }  // namespace csa
 
 using namespace csa;

@@ -170,6 +170,12 @@ struct HeadNormParams {
 __global__ void rmsnorm_rows_kernel(const float* x, const uint16_t* gamma, uint16_t* y, int n, float eps);
 __global__ void head_norm_rope_kernel(HeadNormParams P);
 
+// Host-side checks of csa_indexer_topk's arguments, the workspace aside (api.cu): the
+// workspace-free entry point runs them before it touches its fixed scratch array.
+int check_indexer_topk_args(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
+                            const uint16_t* q_idx, const float* w, const uint16_t* idx_cache, int64_t idx_bstride,
+                            int max_entries, const int32_t* topk_idx);
+
 size_t attn_smem_bytes();
 size_t gemm_smem_bytes();
 size_t indexer_smem_bytes(int stages, int N);

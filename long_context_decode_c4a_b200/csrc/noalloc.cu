@@ -15,7 +15,7 @@
 #include <mutex>
 
 #include "csa.h"
-#include "status.cuh"
+#include "kernels.cuh"
 
 namespace {
 
@@ -49,7 +49,11 @@ extern "C" {
 int csa_indexer_topk_noalloc(int B, int S, int H_I, int d_I, int ratio, int topk, const int32_t* q_pos,
                              const uint16_t* q_idx, const float* w, const uint16_t* idx_cache, int64_t idx_bstride,
                              int max_entries, int32_t* topk_idx, void* stream) {
-  if (B <= 0 || S <= 0 || max_entries <= 0) return CSA_ERR_INVALID_ARG;
+  // Every argument is checked before the fixed array is touched: a refused call writes nothing,
+  // so it cannot clear the status word of another call still running on an unordered stream.
+  if (int rc = csa::check_indexer_topk_args(B, S, H_I, d_I, ratio, topk, q_pos, q_idx, w, idx_cache, idx_bstride,
+                                            max_entries, topk_idx))
+    return rc;
   // The fixed array holds the status word and B*S*max_entries scores; rows longer than one top-k
   // chunk (16384 entries) would need the chunked selection's lists as well, so they are refused.
   const size_t rows = size_t(B) * size_t(S) * size_t(max_entries) * sizeof(float);

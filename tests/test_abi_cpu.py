@@ -197,3 +197,17 @@ def test_calls_with_no_work_are_refused_before_any_launch(lib):
     for kind in (_lib.CSA_WS_INDEXER_TOPK, _lib.CSA_WS_SPARSE_ATTN, _lib.CSA_WS_HCA_ATTN):
         assert lib.csa_workspace_size(kind, 1, 0, 256, 8, ctypes.byref(n)) == _lib.CSA_ERR_INVALID_ARG
 
+
+
+def test_noalloc_refuses_bad_arguments_before_any_cuda_call(lib):
+    """The workspace-free indexer checks its arguments first: on this host without a GPU a refused
+    call returns the argument error, not the CUDA error that touching its device array would give."""
+    p = 1 << 20
+    assert lib.csa_indexer_topk_noalloc(1, 1, 64, 128, 4, 8, p, None, p, p, 1024 * 128, 1024, p,
+                                        None) == _lib.CSA_ERR_INVALID_ARG
+    assert lib.csa_indexer_topk_noalloc(1, 1, 48, 128, 4, 8, p, p, p, p, 1024 * 128, 1024, p,
+                                        None) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_indexer_topk_noalloc(1, 1, 64, 128, 4, 4096, p, p, p, p, 1024 * 128, 1024, p,
+                                        None) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_indexer_topk_noalloc(0, 1, 64, 128, 4, 8, p, p, p, p, 1024 * 128, 1024, p,
+                                        None) == _lib.CSA_ERR_INVALID_ARG

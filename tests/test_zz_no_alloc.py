@@ -50,9 +50,15 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 def test_noalloc_refuses_sizes_beyond_its_array():
     from long_context_decode_c4a_b200 import _lib
     lib = _lib.load()
-    null = None
+    # Nothing is launched for a refused call, so aligned stand-in addresses serve as the tensors.
+    p = 1 << 20
     # 65 queries x 16384 entries of fp32 scores exceed the 4 MiB array; 16385 entries exceed one chunk.
-    assert lib.csa_indexer_topk_noalloc(65, 1, 64, 128, 4, 8, null, null, null, null, 16384 * 128, 16384, null,
-                                        null) == _lib.CSA_ERR_UNSUPPORTED
-    assert lib.csa_indexer_topk_noalloc(1, 1, 64, 128, 4, 8, null, null, null, null, 16385 * 128, 16385, null,
-                                        null) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_indexer_topk_noalloc(65, 1, 64, 128, 4, 8, p, p, p, p, 16384 * 128, 16384, p,
+                                        None) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_indexer_topk_noalloc(1, 1, 64, 128, 4, 8, p, p, p, p, 16385 * 128, 16385, p,
+                                        None) == _lib.CSA_ERR_UNSUPPORTED
+    # Arguments csa_indexer_topk refuses are refused here too, before the array is written.
+    assert lib.csa_indexer_topk_noalloc(1, 1, 48, 128, 4, 8, p, p, p, p, 1024 * 128, 1024, p,
+                                        None) == _lib.CSA_ERR_UNSUPPORTED
+    assert lib.csa_indexer_topk_noalloc(1, 1, 64, 128, 4, 8, p, None, p, p, 1024 * 128, 1024, p,
+                                        None) == _lib.CSA_ERR_INVALID_ARG
