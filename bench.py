@@ -555,35 +555,70 @@ def extra_workloads(args, peaks):
     return res
 
 
-def oracle_decode_time(wl, n_req: int, seed: int = 1):
-    """Seconds the CPU oracle takes for n_req requests of the decode workload."""
+def _oracle_requests(job):
+    """One worker of the CPU oracle's timing (a spawned process with one BLAS thread): draws each
+    request of its seed list untimed, then times the oracle's decode step on it. Returns the summed
+    seconds of the timed steps."""
+    wl, seeds = job
+    from threadpoolctl import threadpool_limits
+
     from oracle import csa_oracle as O
-    small = wl.scaled(B=n_req)
-    inp = O.to_numpy_inputs(make_inputs(small, seed=seed))
-    t = time.perf_counter()
-    for b in range(n_req):
-        if wl.has_indexer:
-            O.csa_decode_request(inp, b, H=wl.H, d=wl.d, W=wl.W, topk=wl.topk)
-        else:
-            O.hca_decode_request(inp, b, H=wl.H, d=wl.d, W=wl.W, ratio=wl.ratio)
-    return time.perf_counter() - t
+    secs = 0.0
+    with threadpool_limits(1):
+        for s in seeds:
+            inp = O.to_numpy_inputs(make_inputs(wl, seed=s))
+            t = time.perf_counter()
+            if wl.has_indexer:
+                O.csa_decode_request(inp, 0, H=wl.H, d=wl.d, W=wl.W, topk=wl.topk)
+            else:
+                O.hca_decode_request(inp, 0, H=wl.H, d=wl.d, W=wl.W, ratio=wl.ratio)
+            secs += time.perf_counter() - t
+    return secs
 
 
-def cpu_threads():
+def host_cores() -> int:
     try:
-        from threadpoolctl import threadpool_info
-        n = [i.get("num_threads", 1) for i in threadpool_info()]
-        return max(n) if n else 1
-    except Exception:  # noqa: BLE001
-        return 1
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # not every platform has an affinity mask
+        return os.cpu_count() or 1
 
 
-def cpu_baseline_decode(wl, budget_s: float = 15.0):
-    one = oracle_decode_time(wl, 1)
-    n = int(max(1, min(wl.B, budget_s / max(one, 1e-3))))
-    secs = oracle_decode_time(wl, n, seed=2)
-    return {"value": n / secs, "unit": "queries/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{n} of the {wl.B} requests of one step ({wl.name}), float64 numpy oracle"}
+class OracleTimer:
+    """The CPU oracle timed on the host cores: independent requests (each drawn with its own seed at
+    the workload's shapes) are spread over one spawned worker process per core, each with one BLAS
+    thread. A batch's time is its makespan: the largest of the workers' summed oracle seconds (the
+    draws of the inputs are not timed)."""
+
+    def __init__(self, wl, cores: int):
+        import multiprocessing
+        self.wl = wl.scaled(B=1)
+        self.cores = max(1, cores)
+        self.pool = multiprocessing.get_context("spawn").Pool(self.cores)
+
+    def time_requests(self, seeds) -> float:
+        jobs = [(self.wl, list(seeds[i::self.cores])) for i in range(self.cores) if seeds[i::self.cores]]
+        return max(self.pool.map(_oracle_requests, jobs, chunksize=1))
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+
+
+def cpu_baseline_decode(wl, budget_s: float = 12.0):
+    """The oracle on a bounded sample of the workload: whole batches of wl.B requests, as many as fit
+    in about budget_s seconds of CPU work spread over the host cores."""
+    cores = min(host_cores(), wl.B)
+    timer = OracleTimer(wl, cores)
+    try:
+        one = timer.time_requests([1])
+        rounds = int(max(1, min(8, budget_s / max(one * wl.B, 1e-3))))
+        seeds = list(range(10, 10 + rounds * wl.B))
+        secs = timer.time_requests(seeds)
+    finally:
+        timer.close()
+    return {"value": len(seeds) / secs, "unit": "queries/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rounds} x {wl.B} requests of {wl.name} (each drawn with its own seed), float64 numpy "
+                      f"oracle, one worker process per core with one BLAS thread; makespan of the oracle's time"}
 
 
 # ------------------------------------------------------------------------------ main
@@ -610,13 +645,17 @@ def main(argv=None):
     wl = WORKLOADS[args.workload]
     if args.batch:
         wl = wl.scaled(B=args.batch)
-    if not wl.is_decode:
-        ap.error("bench.py times the decode workloads; prefill has its own benchmark in the test suite")
-
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # Started without a launcher: start the N ranks here, as torchrun would.
+        return spawn_ranks(args.gpus, sys.argv[1:] if argv is None else list(argv))
     if args.impl == "reference":
+        if not wl.is_decode:
+            ap.error("the reference arm times the decode workloads")
         return run_reference(wl, args)
 
     world, rank, local = dist_setup(args.gpus)
+    if not wl.is_decode:
+        return run_prefill_line(wl, args, world, rank)
     r = run_ours_decode(wl, args, world, rank)
     peaks = load_peaks()
     per_q, reads = decode_bytes(wl)
@@ -674,22 +713,74 @@ def main(argv=None):
     return 0
 
 
+def spawn_ranks(n: int, argv) -> int:
+    """Run this script as n ranks on this node (RANK, LOCAL_RANK, WORLD_SIZE and the rendezvous address
+    set as torchrun sets them); rank 0 prints the JSON line. Returns the largest exit code."""
+    import socket
+    import subprocess
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    procs = []
+    for r in range(n):
+        env = dict(os.environ, RANK=str(r), LOCAL_RANK=str(r), WORLD_SIZE=str(n), LOCAL_WORLD_SIZE=str(n),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        procs.append(subprocess.Popen([sys.executable, os.path.abspath(__file__)] + list(argv), env=env))
+    return max(p.wait() for p in procs)
+
+
+def run_prefill_line(wl, args, world, rank) -> int:
+    """A prefill workload: every rank runs the whole pass on its own GPU (replicas, no collective); the
+    line reports tokens/s over all ranks and the pass's algorithmic tensor FLOPs against the measured
+    dense bf16 peak."""
+    peaks = load_peaks()
+    r = run_prefill(wl, args.steps, args.warmup)
+    ms = max_over_ranks(r["ms"], world)
+    attn_f, idx_f = prefill_ledger(wl)
+    tf = (attn_f + idx_f) / (ms * 1e-3) / 1e12
+    line = {
+        "metric": f"{'CSA' if wl.has_indexer else 'HCA'} prefill tokens/s @{wl.S} tokens; achieved TFLOP/s as % of "
+                  f"B200 dense bf16 peak",
+        "value": world * wl.B * wl.S * 1000.0 / ms, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "requests_per_gpu": wl.B, "tokens": wl.S, "heads": wl.H, "head_dim": wl.d,
+                   "window": wl.W, "topk": wl.topk, "parallelism": f"{world} replica(s), no data-path collective"},
+        "kernels_ms": r["stage_ms"],
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16_tflops"], "peak_source": peaks["source"],
+                     "flops_per_pass": attn_f + idx_f},
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def run_reference(wl, args):
-    """The reference arm: the CPU oracle as it stands, rank 0 only, bounded sample per step."""
+    """The reference arm: the CPU oracle as it stands, rank 0 only, on the host cores; every step is a
+    bounded sample of the workload's requests."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
-    one = oracle_decode_time(wl, 1)
-    per_step = max(1, min(wl.B, int(6.0 / max(one, 1e-3))))
-    total_steps = args.warmup + args.steps
-    while per_step > 1 and total_steps * per_step * one > 150:
-        per_step //= 2
-    for i in range(args.warmup):
-        oracle_decode_time(wl, per_step, seed=10 + i)
-    secs = [oracle_decode_time(wl, per_step, seed=100 + k) for k in range(args.steps)]
+    cores = min(host_cores(), wl.B)
+    timer = OracleTimer(wl, cores)
+    try:
+        one = timer.time_requests([1])
+        per_step = max(1, min(wl.B, int(cores * 2.0 / max(one, 1e-3))))
+        total_steps = args.warmup + args.steps
+        while per_step > 1 and total_steps * per_step * one / cores > 150:
+            per_step //= 2
+        for i in range(args.warmup):
+            timer.time_requests(list(range(1000 + i * per_step, 1000 + (i + 1) * per_step)))
+        secs = [timer.time_requests(list(range(5000 + k * per_step, 5000 + (k + 1) * per_step)))
+                for k in range(args.steps)]
+    finally:
+        timer.close()
     value = per_step * args.steps / sum(secs)
-    cores = cpu_threads()
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000.0 * sum(secs) / args.steps, "higher_is_better": True,
@@ -697,7 +788,8 @@ def run_reference(wl, args):
         "config": {"workload": wl.name, "global_batch": wl.B, "requests_per_gpu": wl.B, "context": wl.ctx,
                    "sample_requests_per_step": per_step},
         "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{per_step} requests of {wl.name} per step, float64 numpy oracle"},
+                         "sample": f"{per_step} requests of {wl.name} per step (each drawn with its own seed), "
+                                   f"float64 numpy oracle, one worker process per core with one BLAS thread"},
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

@@ -1,6 +1,6 @@
 """Build libcsa.so (the CUDA kernels and the C ABI) in-tree for sm_100a.
 
-    python -m long_context_decode_c4a_b200.build [--force] [--debug-bounds]
+    python -m long_context_decode_c4a_b200.build [--force] [-v]
 
 Every .cu file under csrc/ is compiled with nvcc for sm_100a (in parallel) and linked into
 long_context_decode_c4a_b200/libcsa.so with the CUDA runtime linked statically, so the library

@@ -147,3 +147,24 @@ def test_tensor_parallel_indexer_over_two_gloo_ranks():
     assert res[1][1] != "error", res[1]
     assert res[0][1] is True and res[1][1] is True
     assert res[0][2] == (0, 32) and res[1][2] == (32, 64)
+
+
+@pytest.mark.timeout(600)
+def test_bench_starts_its_own_ranks_without_a_launcher():
+    """`python bench.py --gpus 2` without torchrun starts two ranks itself (RANK / WORLD_SIZE set as
+    torchrun sets them); rank 0 alone prints one line, which reports both GPUs. The reference arm runs
+    here, on the CPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--workload", "pro_hca_decode_32k", "--batch", "2", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=500, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [x for x in r.stdout.splitlines() if x.strip()]
+    assert len(lines) == 1, r.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["cpu_baseline"]["cores"] >= 1 and line["value"] > 0
