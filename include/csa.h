@@ -390,6 +390,19 @@ CSA_API int csa_window_projection(int M, int hidden, int d, int rope_dim, float 
  */
 CSA_API int csa_get_device_status(void* ws, void* stream, int* status);
 
+/*
+ * csa_watchdog_selftest -- check the failure path of the kernels' bounded waits (no counterpart in
+ * the pages; failure detection of the library). Every mbarrier wait inside the kernels gives up after
+ * a bounded number of SM cycles (2^30, about half a second), records CSA_ERR_TIMEOUT and the site of
+ * the wait in the status word of `ws` and lets its CTA unwind, instead of hanging the GPU. This call
+ * enqueues one tiny kernel that runs that same wait on a barrier phase nothing completes, giving up
+ * after `limit_cycles` (1 .. 2^30): afterwards csa_get_device_status reports CSA_ERR_TIMEOUT (site
+ * 900 in status word 1) and the context stays usable. Only the status word is written.
+ *   ws/ws_bytes: any workspace of at least 256 bytes, 256-byte aligned (its status word).
+ * Returns CSA_ERR_WORKSPACE / CSA_ERR_INVALID_ARG without launching on bad arguments.
+ */
+CSA_API int csa_watchdog_selftest(void* ws, size_t ws_bytes, long long limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

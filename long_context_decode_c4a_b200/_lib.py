@@ -86,6 +86,7 @@ PROTOTYPES = {
     "csa_decode_fused": (c_int, [POINTER(DecodeArgs), c_void_p]),
     "hca_decode_fused": (c_int, [POINTER(HcaDecodeArgs), c_void_p]),
     "csa_get_device_status": (c_int, [c_void_p, c_void_p, POINTER(c_int)]),
+    "csa_watchdog_selftest": (c_int, [c_void_p, c_size_t, ctypes.c_longlong, c_void_p]),
     "csa_indexer_topk_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
                                          c_void_p, c_int64, c_int, c_void_p, c_void_p]),
     "csa_output_projection": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,

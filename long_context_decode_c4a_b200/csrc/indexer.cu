@@ -240,6 +240,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         if (n < 100) trace_time(status, 600 + (int)n);
         ++n;
       }
+      // After an abort the loads issued last may still be landing in the stages: wait for them
+      // (they complete by themselves) before the CTA can exit. Each of the last min(n, NS) stages
+      // has one load outstanding at most, so its phase parity is unambiguous.
+      for (long long i = n > NS ? n - NS : 0; i < n; ++i)
+        mbar_wait_drain(&sm.k_full[(int)(i % NS)], (uint32_t)((i / NS) & 1), status, 203);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -279,7 +284,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
       }
       // Every MMA issued by this thread completes before TMEM is released.
       mma_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0, abort_flag, status, 214);
+      mbar_wait_drain(&sm.drain, 0, status, 214);
       trace_mark(status, 1, 9);
     }
   } else {

@@ -78,18 +78,18 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar_addr, uint32_t parity) {
 }
 
 // Wait for the phase of `bar` with the given parity to complete. The wait is bounded: after
-// kWaitCycles it records CSA_ERR_TIMEOUT in the device status word, raises the CTA's abort
-// flag and returns false. Once the abort flag is up every later wait returns false at once,
-// so a CTA whose partner role stopped unwinds in bounded time.
+// `limit` SM cycles (kWaitCycles unless given) it records CSA_ERR_TIMEOUT in the device status
+// word, raises the CTA's abort flag and returns false. Once the abort flag is up every later wait
+// returns false at once, so a CTA whose partner role stopped unwinds in bounded time.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, uint32_t site = 0) {
+                                          uint32_t* status, uint32_t site = 0, long long limit = kWaitCycles) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait(addr, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(addr, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       record_status(status, CSA_DEV_TIMEOUT);
       record_site(status, site);
       *abort_flag = 1;
