@@ -252,8 +252,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   cluster_sync();   // the barriers of both CTAs are initialised before any remote access
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  timeline_mark(P.status, kTlAttn, kTlEntry);
   pdl_wait();
   pdl_trigger();
+  timeline_mark(P.status, kTlAttn, kTlReady);
   const int t = P.q_pos[qi];
   if (threadIdx.x == 0) trace_time(status, 0);
 
@@ -688,6 +690,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   if (threadIdx.x == 0) trace_time(status, 255);
   if (warp == kPvWarp) tmem_dealloc(tmem, 512);
+  timeline_mark(P.status, kTlAttn, kTlExit);
 }
 
 size_t attn_smem_bytes() { return 1024 + kStages * kStageBytes + 2 * kXBufs * (size_t)kXBytes + sizeof(AttnSmem); }

@@ -527,9 +527,11 @@ __device__ __forceinline__ void compress_decode_body(const CompressParams& P, in
 __global__ void __launch_bounds__(kCompressThreads) compress_decode_kernel(CompressLaunch L) {
   __shared__ DecodePartial part[kCompressThreads];
   __shared__ float red[kCompressThreads / 32];
+  const CompressParams& P = blockIdx.y != 0 ? L.p[1] : L.p[0];
+  timeline_mark(P.status, kTlCompress, kTlEntry);
   pdl_wait();
   pdl_trigger();
-  const CompressParams& P = blockIdx.y != 0 ? L.p[1] : L.p[0];
+  timeline_mark(P.status, kTlCompress, kTlReady);
   const int b = blockIdx.x;
   if (b >= P.B) return;
   if (P.ratio == 4) {
@@ -539,6 +541,7 @@ __global__ void __launch_bounds__(kCompressThreads) compress_decode_kernel(Compr
     if (P.d == 512) compress_decode_body<128, 512>(P, b, part, red);
     else compress_decode_body<128, 128>(P, b, part, red);
   }
+  timeline_mark(P.status, kTlCompress, kTlExit);
 }
 
 // Final state of a multi-token segment: one CTA per request, reads before writes.

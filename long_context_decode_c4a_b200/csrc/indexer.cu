@@ -200,8 +200,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  timeline_mark(P.status, kTlIndexer, kTlEntry);
   pdl_wait();
   pdl_trigger();
+  timeline_mark(P.status, kTlIndexer, kTlReady);
   if (threadIdx.x == 0) trace_time(P.status, 599);
 
   const long long total = P.total_items;
@@ -333,6 +335,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   if (threadIdx.x == 0) trace_mark(status, 3, 2);
   if (warp == 1) tmem_dealloc(tmem, acc_cols);
   if (threadIdx.x == 32) trace_mark(status, 3, 3);
+  timeline_mark(status, kTlIndexer, kTlExit);
 }
 
 size_t indexer_smem_bytes(int stages, int N) {

@@ -69,4 +69,27 @@ __device__ __forceinline__ void trace_time(uint32_t* status, int idx) {
 #endif
 }
 
+// Step timeline for profiling builds (-DCSA_STEP_TIMELINE): thread 0 of every CTA folds the
+// %globaltimer (ns) at kernel entry (min over CTAs), after its dependency wait (min) and at its end
+// (max) into uint64 words 8 + 3*kernel + {0, 1, 2} of the status area (bytes 64..255 of the
+// workspace, which the caller presets to ~0 / ~0 / 0). Kernel ids: see TimelineKernel. Compiled out
+// otherwise.
+enum TimelineKernel { kTlCompress = 0, kTlIndexer = 1, kTlTopk = 2, kTlTopkMerge = 3, kTlAttn = 4 };
+enum TimelineWhat { kTlEntry = 0, kTlReady = 1, kTlExit = 2 };
+__device__ __forceinline__ void timeline_mark(uint32_t* status, int kernel, int what) {
+#ifdef CSA_STEP_TIMELINE
+  if (status != nullptr && threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    unsigned long long* w = reinterpret_cast<unsigned long long*>(status) + 8 + 3 * kernel + what;
+    if (what == kTlExit) atomicMax(w, t);
+    else atomicMin(w, t);
+  }
+#else
+  (void)status;
+  (void)kernel;
+  (void)what;
+#endif
+}
+
 }  // namespace csa

@@ -379,11 +379,14 @@ __device__ void topk_chunk(const TopkParams& P, TopkRegShared& sh) {
 // the candidate buffers for topk_merge_kernel.
 __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) {
   __shared__ TopkRegShared sh;
+  timeline_mark(P.status, kTlTopk, kTlEntry);
   pdl_wait();
   pdl_trigger();
+  timeline_mark(P.status, kTlTopk, kTlReady);
   // Rows of <= kTopkShortRow entries hold 8 keys per thread, chunks of kTopkChunk entries 16.
   if (P.max_entries <= kTopkShortRow) topk_chunk<kTopkShortThreads, kTopkShortRow / kTopkShortThreads>(P, sh);
   else topk_chunk<kTopkThreads, kTopkChunk / kTopkThreads>(P, sh);
+  timeline_mark(P.status, kTlTopk, kTlExit);
 }
 
 // One CTA per query with more than one chunk: top-k over the union of the chunks' lists. The
@@ -392,8 +395,10 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
 __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) {
   __shared__ TopkShared sh;
   __shared__ int cnts[kTopkMaxChunks];
+  timeline_mark(P.status, kTlTopkMerge, kTlEntry);
   pdl_wait();
   pdl_trigger();
+  timeline_mark(P.status, kTlTopkMerge, kTlReady);
   const int q = blockIdx.x;
   const int t = P.q_pos[q];
   int E = (t + 1) / P.ratio;
@@ -412,6 +417,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) 
   int32_t* out = P.out + (long long)q * P.topk;
   const uint32_t cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = ci[i]; }, sh);
   for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
+  timeline_mark(P.status, kTlTopkMerge, kTlExit);
 }
 
 }  // namespace csa
