@@ -142,11 +142,11 @@ int device_info(DeviceInfo** out) {
 
 // ---- workspace layout
 struct IdxWs {
-  size_t scores_off, cand_key_off, cand_idx_off, cand_cnt_off, total;
+  size_t scores_off, cand_key_off, cand_idx_off, cand_cnt_off, flags_off, total;
   int max_chunks;
 };
 
-IdxWs indexer_ws_layout(long long queries, int max_entries, int topk) {
+IdxWs indexer_ws_layout(long long queries, int max_entries, int topk, bool with_flags = false) {
   IdxWs w{};
   size_t off = kStatusBytes;
   w.scores_off = off;
@@ -158,6 +158,8 @@ IdxWs indexer_ws_layout(long long queries, int max_entries, int topk) {
   off = round_up(off + (size_t)queries * w.max_chunks * topk * 4, 256);
   w.cand_cnt_off = off;
   off = round_up(off + (size_t)queries * w.max_chunks * 4, 256);
+  w.flags_off = off;                       // fused decode step: per-request index-entry flags
+  if (with_flags) off = round_up(off + (size_t)queries * 4, 256);
   w.total = off;
   return w;
 }
@@ -287,11 +289,11 @@ int check_indexer_args(const IndexerArgs& a, bool scores = true, bool select = t
 // serve the tensor-parallel indexer: partial scores per head shard, a sum across ranks, then the
 // selection.
 int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* ev = nullptr, bool run_scores = true,
-                     bool run_select = true) {
+                     bool run_select = true, const CompressLaunch* fuse = nullptr) {
   DeviceInfo* dev;
   if (int rc = device_info(&dev)) return rc;
   const long long queries = (long long)a.B * a.S;
-  const IdxWs L = indexer_ws_layout(queries, a.max_entries, run_select ? a.topk : 1);
+  const IdxWs L = indexer_ws_layout(queries, a.max_entries, run_select ? a.topk : 1, fuse != nullptr);
   const size_t need = run_select ? (a.scores_opt ? L.total - (L.cand_key_off - L.scores_off) : L.total) : kStatusBytes;
   if (int rc = check_ws(a.ws, a.ws_bytes, need)) return rc;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
@@ -312,9 +314,11 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
     P.tiles_per_group = (a.max_entries + 127) / 128;
     P.total_items = (long long)a.B * P.groups_per_req * P.tiles_per_group;
     P.rows_per_req = a.idx_bstride / a.d_I;
+    const bool fused = fuse != nullptr;
     int stages = kIdxMaxStages;
-    while (stages > 2 && indexer_smem_bytes(stages, P.N) > (size_t)dev->max_smem) --stages;
-    CSA_CHECK_SUP(indexer_smem_bytes(stages, P.N) <= (size_t)dev->max_smem, "shared memory too small for the indexer");
+    while (stages > 2 && indexer_smem_bytes(stages, P.N, fused) > (size_t)dev->max_smem) --stages;
+    CSA_CHECK_SUP(indexer_smem_bytes(stages, P.N, fused) <= (size_t)dev->max_smem,
+                  "shared memory too small for the indexer");
     P.stages = stages;
     P.n_acc = (4 * P.N <= 512) ? 4 : 2;
     int cols = 32;
@@ -329,16 +333,23 @@ int run_indexer_topk(const IndexerArgs& a, cudaStream_t st, cudaEvent_t const* e
     CUtensorMap map_k, map_q;
     if (int rc = make_map_2d(&map_k, a.idx_cache, 128, (uint64_t)a.B * P.rows_per_req, 128, 64, 128)) return rc;
     if (int rc = make_map_2d(&map_q, a.q_idx, 128, (uint64_t)queries * a.H_I, 128, 64, (uint32_t)P.N)) return rc;
-    const size_t smem = indexer_smem_bytes(stages, P.N);
+    const size_t smem = indexer_smem_bytes(stages, P.N, fused);
     const dim3 grid((unsigned)std::min<long long>(P.total_items, dev->sms));
+    IndexerFuse F{};
+    if (fused) {
+      F.njobs = 2 * a.B;
+      F.B = a.B;
+      F.flags = reinterpret_cast<uint32_t*>(ws + L.flags_off - shift);
+      F.L = *fuse;
+    }
     cudaError_t e = cudaSuccess;
     switch (a.H_I) {
-      case 4: e = launch_pdl(indexer_kernel<4>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-      case 8: e = launch_pdl(indexer_kernel<8>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-      case 16: e = launch_pdl(indexer_kernel<16>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-      case 32: e = launch_pdl(indexer_kernel<32>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-      case 64: e = launch_pdl(indexer_kernel<64>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
-      default: e = launch_pdl(indexer_kernel<128>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P); break;
+      case 4: e = launch_pdl(indexer_kernel<4>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P, F); break;
+      case 8: e = launch_pdl(indexer_kernel<8>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P, F); break;
+      case 16: e = launch_pdl(indexer_kernel<16>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P, F); break;
+      case 32: e = launch_pdl(indexer_kernel<32>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P, F); break;
+      case 64: e = launch_pdl(indexer_kernel<64>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P, F); break;
+      default: e = launch_pdl(indexer_kernel<128>, grid, dim3(kIdxThreads), smem, st, map_k, map_q, P, F); break;
     }
     CSA_CUDA(e);
   }
@@ -526,7 +537,7 @@ int csa_workspace_size(int kind, int B, int S, int max_entries, int topk, size_t
     case CSA_WS_INDEXER_TOPK:
     case CSA_WS_DECODE_FUSED:
       CSA_CHECK_ARG(topk > 0, "topk must be positive");
-      *bytes = indexer_ws_layout((long long)B * S, max_entries, topk).total;
+      *bytes = indexer_ws_layout((long long)B * S, max_entries, topk, kind == CSA_WS_DECODE_FUSED).total;
       return CSA_OK;
     case CSA_WS_SPARSE_ATTN:
     case CSA_WS_HCA_ATTN:
@@ -803,7 +814,7 @@ int csa_decode_fused(const csa_decode_args* a, void* stream) {
               a->ring_bstride, a->ring_cap, a->window, a->cache, a->cache_bstride, a->max_entries, a->topk_idx,
               a->topk, a->sink, a->out, a->out_is_f32, a->ws, a->ws_bytes};
   if (int rc = check_attn_args(aa, true)) return rc;
-  const IdxWs L = indexer_ws_layout(a->B, a->max_entries, a->topk);
+  const IdxWs L = indexer_ws_layout(a->B, a->max_entries, a->topk, true);
   if (int rc = check_ws(a->ws, a->ws_bytes, L.total)) return rc;
 
   uint32_t* status = static_cast<uint32_t*>(a->ws);
@@ -817,10 +828,11 @@ int csa_decode_fused(const csa_decode_args* a, void* stream) {
   CL.p[1] = compress_params(&idx_cfg, a->B, 1, a->pos, a->idx_kv, a->idx_score, a->idx_gamma, a->idx_state_kv,
                             a->idx_state_score, a->idx_cache, a->idx_bstride, a->max_entries, nullptr, status);
   cudaEvent_t const* ev = reinterpret_cast<cudaEvent_t const*>(a->stage_events);
+  // The compressor step of both streams runs inside the indexer launch (its epilogue warps, before
+  // their first tile); the "compress" stage interval is therefore empty.
   if (ev) CSA_CUDA(cudaEventRecord(ev[0], st));
-  if (int rc = launch_compress(CL, 2, a->B, 1, a->ratio, st)) return rc;
   if (ev) CSA_CUDA(cudaEventRecord(ev[1], st));
-  if (int rc = run_indexer_topk(ia, st, ev ? ev + 2 : nullptr)) return rc;
+  if (int rc = run_indexer_topk(ia, st, ev ? ev + 2 : nullptr, true, true, &CL)) return rc;
   if (int rc = run_attn(aa, true, st)) return rc;
   if (ev) CSA_CUDA(cudaEventRecord(ev[4], st));
   return CSA_OK;

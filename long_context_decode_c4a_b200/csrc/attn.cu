@@ -57,19 +57,27 @@ constexpr int kProducers = 128;               // warps 0..3
 constexpr int kQkWarp0 = 4;                   // warps 4, 5: score MMAs of even / odd tiles
 constexpr int kPvWarp = 6;                    // PV MMAs; owns TMEM
 constexpr int kSendWarp0 = 7;                 // warps 7..10: send partial scores
-constexpr int kSoftWarp0 = 11;                // warps 11..14: softmax
+constexpr int kSoftWarp0 = 11;                // warps 11..14: softmax of even tiles, 15..18 of odd tiles
 constexpr int kRoleThreads = 128;
 constexpr int kTile = 32;                     // candidates per tile
-constexpr int kStages = 8;
+// Gather stages and exchange buffers (build-time tuning knobs; attn_smem_bytes() reports the shared
+// memory they take, which the launch checks).
+#ifndef CSA_ATTN_STAGES
+#define CSA_ATTN_STAGES 8
+#endif
+#ifndef CSA_ATTN_XBUFS
+#define CSA_ATTN_XBUFS 2
+#endif
+constexpr int kStages = CSA_ATTN_STAGES;
 constexpr int kSBufs = 2;                     // partial-score tiles in TMEM
 constexpr uint32_t kStageBytes = 16 * 1024;   // 32 rows x 256 dims of bf16
 constexpr uint32_t kBlockBytes = 4096;        // one 64-dim block of a stage: [32 rows][128 B]
 constexpr uint32_t kXBytes = 16 * 1024;       // 128 heads x 32 fp32 partial scores
 constexpr uint32_t kOutRow = 512 + 16;        // bf16 output staging: 256 dims per head row, padded
-constexpr int kXBufs = 2;                     // exchange buffers each way
+constexpr int kXBufs = CSA_ATTN_XBUFS;        // exchange buffers each way
 constexpr int kPBufs = 2;                     // P tiles in TMEM
 
-static_assert(kAttnThreads == 32 * (kSoftWarp0 + 4), "warp roles");
+static_assert(kAttnThreads == 32 * (kSoftWarp0 + 8), "warp roles");
 static_assert(kAttnMaxCands % kTile == 0, "candidate capacity");
 static_assert(kXBufs >= 2, "exchange buffers");
 static_assert(kXBufs * 2 * kXBytes >= 64 * 1024, "Q[:, half] is staged over the exchange buffers");
@@ -89,6 +97,8 @@ struct AttnSmem {
   uint64_t x_empty[kXBufs][4];        // the other CTA consumed the 4 KB this warp sent last
   uint64_t x_staged[kXBufs][4];       // this CTA's 4 KB is staged in the outgoing buffer
   uint64_t x_own[kXBufs][4];          // this CTA's softmax warp read its staged 4 KB
+  uint64_t hand[2][4];                // softmax group g published the running max after its tile (quadrant q)
+  uint64_t b_done;                    // softmax group 1 left its part of the denominator in l_b / m_b
   uint64_t epi;                       // the softmax warps published 1/l
   uint64_t drain[3];
   uint32_t tmem_base;
@@ -99,6 +109,8 @@ struct AttnSmem {
   uint32_t scan[kProducers / 32];
   float rope_cs[kMaxRopePairs][2];
   float inv_l[128];
+  float m_hand[4][32];                // running max handed from one softmax group to the other
+  float l_b[128], m_b[128];           // softmax group 1's part of the denominator and its max
   uint32_t mask[kAttnMaxCands / kTile];
   uint32_t list[kAttnMaxCands];
 };
@@ -143,6 +155,11 @@ __device__ __forceinline__ uint32_t producer_scan(uint32_t v, uint32_t* scan, ui
   named_bar_sync(2, kProducers);
   total = tot;
   return off + inc - v;
+}
+
+// Fine-grained timeline of tile j (debugging builds only): slot 0..15 of word 2000 + 16 j.
+__device__ __forceinline__ void trace_tile(uint32_t* status, int j, int slot) {
+  if (j < 40) trace_time(status, 2000 + 16 * j + slot);
 }
 
 // O[:, half] / l for columns [c0, c0 + 32 nchunks) of this CTA's 256 dims of row h (the global dims
@@ -238,6 +255,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       }
     }
     mbar_init(&sm.epi, kRoleThreads);
+    for (int gg = 0; gg < 2; ++gg)
+      for (int q = 0; q < 4; ++q) mbar_init(&sm.hand[gg][q], 32);
+    mbar_init(&sm.b_done, kRoleThreads);
     for (int i = 0; i < 3; ++i) mbar_init(&sm.drain[i], 1);
     sm.abort_flag = 0;
     sm.bad = 0;
@@ -291,7 +311,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         const char* src = ((e & kFromCache) ? cache_base : ring_base) + (size_t)(e & kRowMask) * 1024 + w * 16;
         cp_async_16(st + (w >> 3) * kBlockBytes + sw128_offset(r, w & 7), src);
       }
-      cp_async_commit();
+      cp_async_arrive_noinc(&sm.kv_full[tile % kStages]);
     };
     // Tiles made only of window rows are known now: their gathers start before the compressed
     // entries are read.
@@ -351,44 +371,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       trace_time(status, 1);
     }
 
-    // Gathers: tile j -> stage j % kStages. The loop issues the next tile whenever its stage is free
-    // and otherwise waits for its oldest tile in flight and announces it (kv_full), so tiles are
-    // announced as soon as they land while up to kStages tiles are in flight. Each thread runs the
-    // loop on its own (its decisions may differ from other threads'); every thread arrives once
-    // per tile.
-    int next = w_tiles, ann = 0;
-    while (ann < J) {
-      bool go = next < J;
-      if (go && next >= kStages) {
-        uint64_t* empty = &sm.buf_free[next % kStages];
-        const uint32_t par = (uint32_t)((next / kStages - 1) & 1);
-        if (next > ann) {
-          go = mbar_test(smem_u32(empty), par);
-        } else if (!mbar_wait(empty, par, abort_flag, status, 102)) {
-          break;
-        }
-      }
-      if (go) {
-        issue(next);
-        ++next;
-        continue;
-      }
-      switch (next - ann) {  // groups committed after the oldest tile in flight
-        case 1: cp_async_wait<0>(); break;
-        case 2: cp_async_wait<1>(); break;
-        case 3: cp_async_wait<2>(); break;
-        case 4: cp_async_wait<3>(); break;
-        case 5: cp_async_wait<4>(); break;
-        case 6: cp_async_wait<5>(); break;
-        case 7: cp_async_wait<6>(); break;
-        default: cp_async_wait<7>(); break;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&sm.kv_full[ann % kStages]);
-      if (pt == 0 && ann < 60) trace_time(status, 2 + ann);
-      ++ann;
+    // Gathers: tile j -> stage j % kStages, issued in order as soon as the stage is free (PV of tile
+    // j - kStages completed). Each thread's copies arrive on kv_full by themselves when they land
+    // (cp.async.mbarrier.arrive), so issuing never waits for a tile in flight; the consumers order
+    // the landed bytes before their tensor-core reads with a proxy fence.
+    for (int next = w_tiles; next < J; ++next) {
+      if (next >= kStages &&
+          !mbar_wait(&sm.buf_free[next % kStages], (uint32_t)((next / kStages - 1) & 1), abort_flag, status, 102))
+        break;
+      issue(next);
+      if (pt == 0 && next < 60) trace_time(status, 2 + next);
     }
-    cp_async_wait<0>();  // after an abort: let the copies land before teardown
+    cp_async_wait_all();  // after an abort: let the copies land before teardown
   } else if (warp < kPvWarp) {
     // ------------------------------------------------------------ score MMAs: tiles j = w, w+2, ...
     if (lane == 0) {
@@ -402,7 +396,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         // Score tile sb is rewritten only once the senders have loaded tile j - kSBufs.
         if (j >= kSBufs && !mbar_wait(&sm.s_rd[sb], (uint32_t)((j / kSBufs - 1) & 1), abort_flag, status, 117))
           break;
+        trace_tile(status, j, 0);
         if (!mbar_wait(&sm.kv_full[s], (uint32_t)((j / kStages) & 1), abort_flag, status, 114)) break;
+        fence_proxy_async_smem();  // the gathered rows (written by cp.async) before the MMAs read them
         tc_fence_after();
         if (j < 60) trace_time(status, 64 + j);
         const uint32_t kbase = smem_u32(stage0 + (size_t)s * kStageBytes);
@@ -413,6 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           mma_ts(d_s, tmem + 8 * ks, bdesc, idesc_qk, ks > 0 ? 1u : 0u);
         }
         mma_commit(&sm.s_full[sb]);
+        trace_tile(status, j, 2);
       }
       // Every MMA issued above completes on its own; wait for them before TMEM is released.
       mma_commit(&sm.drain[w]);
@@ -427,6 +424,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       for (int j = 0; j < J; ++j) {
         const int pb = j % kPBufs;
         if (!mbar_wait(&sm.p_full[pb], (uint32_t)((j / kPBufs) & 1), abort_flag, status, 115)) break;
+        trace_tile(status, j, 3);
+        fence_proxy_async_smem();  // the gathered rows of the tile before the MMAs read them
         tc_fence_after();
         const uint32_t vbase = smem_u32(stage0 + (size_t)(j % kStages) * kStageBytes);
         const uint32_t pcol = tmem + 128 + kTile * (kSBufs + pb);
@@ -448,13 +447,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   } else {
     // ------------------------------------------------------------ senders (7..10), softmax (11..14)
     const bool sender = warp < kSoftWarp0;
+    const bool softB = warp >= kSoftWarp0 + 4;  // second softmax group (odd tiles)
     const int quad = warp & 3;             // TMEM lane quadrant
     const int h = quad * 32 + lane;        // head = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const int rt = threadIdx.x - (sender ? kSendWarp0 : kSoftWarp0) * 32;  // 0..127 within the role
+    const int rt = threadIdx.x - (sender ? kSendWarp0 : (softB ? kSoftWarp0 + 4 : kSoftWarp0)) * 32;  // 0..127 within the role
     // Q[:, half] -> TMEM columns [0, 128): blocks 0-1 by the senders, 2-3 by the softmax warps.
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag, status, 121));
-    if (ok) {
+    bool ok = softB || __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0, abort_flag, status, 121));
+    if (ok && !softB) {
 #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         const int kb = (sender ? 0 : 2) + kk;
@@ -471,17 +471,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
       }
       tmem_wait_st();
     }
-    tc_fence_before();
-    mbar_arrive(&sm.q_done);
+    if (!softB) {
+      tc_fence_before();
+      mbar_arrive(&sm.q_done);
+    }
     // Inverse-RoPE table for position t.
     const int npairs = P.rope_dim / 2;
-    if (!sender && rt < npairs) {
+    if (!sender && !softB && rt < npairs) {
       float cs, sn;
       rope_cos_sin(t, P.inv_freq[rt], &cs, &sn);
       sm.rope_cs[rt][0] = cs;
       sm.rope_cs[rt][1] = -sn;
     }
-    named_bar_sync(1, 2 * kRoleThreads);   // the Q staging area is no longer read
+    if (!softB) named_bar_sync(1, 2 * kRoleThreads);   // the Q staging area is no longer read
     ok = __all_sync(0xffffffffu, ok && mbar_wait(&sm.list_ready, 0, abort_flag, status, 122));
     const int J = ok ? sm.n_tiles : 0;
     // Tile j travels through exchange buffer c = j % kXBufs; phase (j / kXBufs) & 1 of x_full /
@@ -498,10 +500,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         const int c = j % kXBufs, sb = j % kSBufs;
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (uint32_t)((j / kSBufs) & 1), abort_flag, status, 123)))
           break;
+        if (rt == 0) trace_tile(status, j, 5);
         tc_fence_after();
         uint32_t v[32];
         tmem_ld32(tmem + lane_addr + 128 + kTile * sb, v);
         tmem_wait_ld();
+        if (rt == 0) trace_tile(status, j, 6);
         // The partial scores are read: the score MMAs of tile j + kSBufs may overwrite them.
         tc_fence_before();
         mbar_arrive(&sm.s_rd[sb]);
@@ -510,6 +514,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         if (!__all_sync(0xffffffffu, mbar_wait_cluster(&sm.x_empty[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag,
                                                         status, 126)))
           break;
+        if (rt == 0) trace_tile(status, j, 7);
         if (j >= kXBufs &&
             !__all_sync(0xffffffffu, mbar_wait(&sm.x_own[c][quad], (uint32_t)((j / kXBufs - 1) & 1), abort_flag, status, 130)))
           break;
@@ -526,36 +531,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         }
       }
     } else {
-      // Every incoming buffer is free: arm them, then let the other CTA send.
-      if (lane == 0)
-        for (int c = 0; c < kXBufs; ++c) {
+      // Softmax warps: group 0 (warps 11..14) takes the even tiles, group 1 (warps 15..18) the odd
+      // ones; each owns the 32 heads of its quadrant. The running max passes from the group that
+      // finished tile j - 1 to the one taking tile j through hand[group][quad] (one mbarrier phase
+      // per tile, 32 arrivals: the publishing warp's lanes).
+      const int g = softB ? 1 : 0;
+      if (!softB && lane == 0)
+        for (int c = 0; c < kXBufs; ++c) {  // every incoming buffer is free: arm them, let the other CTA send
           mbar_arrive_expect_tx(&sm.x_full[c][quad], kXBytes / 4);
           mbar_arrive_remote_relaxed(xempty_peer + 32 * c);
         }
       const float sl = (h < P.H) ? P.sink[h] * 1.4426950408889634f : 0.f;
-      float m_used = sl;  // running max in log2 units (starts at the sink)
-      float l = 1.f;      // running denominator; the sink contributes exp2(sl - m_used) = 1
-      // p_free[i % kPBufs] completes once per PV(i). A parity wait for PV(i) is unambiguous while
-      // PV(i - kPBufs) has been observed and PV(i + kPBufs) cannot have completed, so PV
-      // completions are observed in order: PV(j - 2) before P of tile j is stored (its P tile is
-      // then free; PV(j) is not issued yet), PV(j - 1) before a rescale, PV(J - 1) before the
-      // epilogue.
+      float m_used = sl;         // running max in log2 units (starts at the sink), as this group last saw it
+      float l = softB ? 0.f : 1.f;  // this group's part of the denominator, relative to m_used; group 0
+                                 // holds the sink's exp2(sl - m_used) = 1
+      // p_free[i % 2] completes once per PV(i): p_free[g] counts the PVs of group g's tiles. A parity
+      // wait for PV(i) is unambiguous while the barrier's previous phase (PV(i - 2)) has completed and
+      // its next one (PV(i + 2)) cannot have. Each group therefore waits only for: PV(j - 2) of its
+      // own previous tile before storing P of tile j (it waited for PV(j - 4) before storing P(j - 2);
+      // PV(j) is not issued yet); before a rescale, that one and then PV(j - 1) of the other group
+      // (PV completions are in issue order, so PV(j - 3) is done once PV(j - 2) is, and PV(j + 1)
+      // waits for the running max this group has not published yet); group 0 waits for the last PVs
+      // before the epilogue the same way.
       static_assert(kPBufs == 2, "P tile j is stored once PV(j - 2) completed");
-      int pv_seen = 0;  // PV(0 .. pv_seen-1) observed complete
-      auto observe_pv = [&](int upto) -> bool {  // observe PV(pv_seen .. upto-1)
-        for (; pv_seen < upto; ++pv_seen)
-          if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_free[pv_seen % kPBufs], (uint32_t)((pv_seen / kPBufs) & 1),
-                                                 abort_flag, status, 124)))
-            return false;
-        return true;
+      auto wait_pv = [&](int i) -> bool {
+        return i < 0 || __all_sync(0xffffffffu, mbar_wait(&sm.p_free[i % kPBufs], (uint32_t)((i / kPBufs) & 1),
+                                                           abort_flag, status, 124));
       };
-      for (; j < J; ++j) {
+      bool done = true;
+      for (j = g; j < J; j += 2) {
         const int c = j % kXBufs;
         // This CTA's partial scores of the tile (staged by the sender) and the other CTA's.
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_staged[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag, status, 128)))
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_staged[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag, status, 128))) {
+          done = false;
           break;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_full[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag, status, 127)))
+        }
+        if (rt == 0) trace_tile(status, j, 10);
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.x_full[c][quad], (uint32_t)((j / kXBufs) & 1), abort_flag, status, 127))) {
+          done = false;
           break;
+        }
         if (rt == 0 && j < 60) trace_time(status, 400 + j);
         // S = S_0 + S_1 (the same sum in both CTAs), scaled to log2 units; padding -> -inf.
         const uint8_t* xi = xin + c * kXBytes;
@@ -597,15 +612,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           mbar_arrive(&sm.x_own[c][quad]);
         }
         if (rt == 0 && j < 60) trace_time(status, 500 + j);
+        // The running max after tile j - 1, from the other group (it only grows: this group's part
+        // of the denominator follows it).
+        if (j > 0) {
+          const int pj = j - 1;  // published by group 1 - g as its (pj / 2)-th tile
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.hand[1 - g][quad], (uint32_t)((pj / 2) & 1), abort_flag, status,
+                                                 131))) {
+            done = false;
+            break;
+          }
+          const float mp = sm.m_hand[quad][lane];
+          if (mp != m_used) {
+            l *= exp2f(m_used - mp);
+            m_used = mp;
+          }
+        }
         // Lazy rescale: only when this tile raises the row max by more than 2^8. The TMEM accesses
         // are warp-collective, so the whole warp takes the branch if any lane needs it (lanes that do
         // not need it scale by 1).
+        if (rt == 0) trace_tile(status, j, 12);
         const bool need = mt > m_used + 8.f;
         const float alpha = need ? exp2f(m_used - mt) : 1.f;
         if (__any_sync(0xffffffffu, need)) {
           if (j > 0) {
             // O holds PV(0..j-1): wait for PV(j-1), then scale the rows of this warp.
-            if (!observe_pv(j)) break;
+            if (!wait_pv(j - 2) || !wait_pv(j - 1)) {
+              done = false;
+              break;
+            }
             tc_fence_after();
 #pragma unroll 1
             for (int cc = 0; cc < 8; ++cc) {
@@ -618,11 +652,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
               tmem_st32(oa, o);
             }
             tmem_wait_st();
+            tc_fence_before();
           }
           if (need) {
             l *= alpha;
             m_used = mt;
           }
+        }
+        // Publish the running max for tile j + 1 (taken by the other group).
+        if (j + 1 < J) {
+          sm.m_hand[quad][lane] = m_used;
+          mbar_arrive(&sm.hand[g][quad]);
         }
         // P = P_hi + P_lo, both bf16, in P tile j % kPBufs: P_hi in columns [0,16), P_lo in
         // [16,32). P_hi is p truncated to bf16 (the high half of its bits); P_lo = p - P_hi is exact
@@ -644,7 +684,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
           for (int e = 0; e < w; ++e) ps[e] += ps[e + w];
         l += ps[0];
         // P tile j % kPBufs was read by PV(j - kPBufs).
-        if (!observe_pv(j - 1)) break;
+        if (rt == 0) trace_tile(status, j, 13);
+        if (!wait_pv(j - 2)) {
+          done = false;
+          break;
+        }
+        if (rt == 0) trace_tile(status, j, 14);
         tc_fence_after();
         const uint32_t pa = tmem + lane_addr + 128 + kTile * (kSBufs + j % kPBufs);
         tmem_st16(pa, phi);
@@ -652,13 +697,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[j % kPBufs]);
+        if (lane == 0 && j < 40) trace_time(status, 3000 + 4 * j + quad);
         if (rt == 0 && j < 60) trace_time(status, 128 + j);
       }
-      if (j == J && !observe_pv(J)) j = -1;
-      sm.inv_l[h] = 1.f / l;
+      if (softB) {
+        // Group 1 hands its part of the denominator (and the max it is relative to) to group 0.
+        sm.l_b[h] = l;
+        sm.m_b[h] = m_used;
+        mbar_arrive(&sm.b_done);
+        j = done ? J : -1;
+      } else {
+        // Every PV completed: this group's last one, then (when the last tile was group 1's) PV(J - 1).
+        const int last0 = ((J - 1) & ~1);
+        if (done && J > 0 && (!wait_pv(last0) || !wait_pv(J - 1))) done = false;
+        if (done && !__all_sync(0xffffffffu, mbar_wait(&sm.b_done, 0, abort_flag, status, 132))) done = false;
+        if (done) {
+          const float lb = sm.l_b[h], mb = sm.m_b[h];
+          const float mf = fmaxf(m_used, mb);  // the last published max (it only grows)
+          l = (l != 0.f ? l * exp2f(m_used - mf) : 0.f) + (lb != 0.f ? lb * exp2f(mb - mf) : 0.f);
+        }
+        sm.inv_l[h] = 1.f / l;
+        j = done ? J : -1;
+      }
     }
-    // Epilogue: O / l, inverse RoPE on the rotated dims, store. The softmax warps take O columns
-    // [0, 128) of their rows, the senders [128, 256).
+    // Epilogue: O / l, inverse RoPE on the rotated dims, store. The softmax warps of group 0 take O
+    // columns [0, 128) of their rows, the senders [128, 256); group 1 has finished.
+    if (!softB) {
     bool fin;
     if (sender) {
       fin = __all_sync(0xffffffffu, j == J && J > 0 && mbar_wait(&sm.epi, 0, abort_flag, status, 125));
@@ -682,6 +746,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         bulk_commit();
         bulk_wait_read_all();
       }
+    }
     }
   }
   __syncwarp();

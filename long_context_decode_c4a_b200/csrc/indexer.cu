@@ -18,6 +18,7 @@
 // split into contiguous ranges per CTA so the Q tile of a group is loaded once per CTA. Tiles
 // past the group's last visible entry are skipped by every role alike.
 
+#include "compress_decode.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -101,6 +102,28 @@ struct ItemIter {
   }
 };
 
+// Wait (bounded) until another CTA raises *flag, then clear it for the next call and order the
+// loads that follow through the tensor-memory-access (async) proxy after what the flag published.
+__device__ __forceinline__ bool wait_flag_and_clear(uint32_t* flag, volatile int* abort_flag, uint32_t* status,
+                                                    uint32_t site) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v != 0u) break;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      record_status(status, CSA_DEV_TIMEOUT);
+      record_site(status, site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(0u) : "memory");
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
 struct IdxSmem {
   uint64_t k_full[kIdxMaxStages], k_empty[kIdxMaxStages];
   uint64_t q_full[2], q_empty[2];
@@ -154,7 +177,7 @@ __device__ __forceinline__ void epilogue_tile(const IndexerParams& P, const floa
 template <int HI>
 __global__ void __launch_bounds__(kIdxThreads, 1)
     indexer_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
-                   IndexerParams P) {
+                   IndexerParams P, IndexerFuse F) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int NS = P.stages;
@@ -166,6 +189,10 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   // Per epilogue group: w of the group's current queries (N floats) and their visible entries.
   float* w_arr = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(IdxSmem));
   int* vis_arr = reinterpret_cast<int*>(w_arr + 2 * N);
+  // Fused decode compression: the body's partials and reduction scratch.
+  DecodePartial* part = reinterpret_cast<DecodePartial*>(
+      (reinterpret_cast<uintptr_t>(vis_arr + 2 * N) + 15) & ~uintptr_t(15));
+  float* red = reinterpret_cast<float*>(part + kCompressThreads);
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -233,6 +260,11 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         const int st = (int)(n % NS);
         const uint32_t ph = (uint32_t)((n / NS) & 1);
         if (!mbar_wait(&sm.k_empty[st], ph ^ 1, abort_flag, status, 202)) break;
+        if (F.njobs > 0) {
+          // The tile holding the request's last visible entry waits for this step's index entry.
+          const int vis = visible_of(P, c.b, c.qg * P.QG);
+          if (vis > 0 && c.et == (vis - 1) / 128 && !wait_flag_and_clear(&F.flags[c.b], abort_flag, status, 204)) break;
+        }
         mbar_arrive_expect_tx(&sm.k_full[st], 32768);
         const int krow = (int)((long long)c.b * P.rows_per_req + (long long)c.et * 128);
         uint8_t* dst = k_tiles + (size_t)st * 32768;
@@ -293,6 +325,22 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     // ---------------------------------------------------------------- epilogue (warps 2..9)
     // Two groups of four warps take alternate work items (group g: items n with n % 2 == g), each
     // group covering the four TMEM lane quadrants.
+    if (F.njobs > 0) {
+      // The step's compression jobs first (index streams before main streams); named barriers 5-7.
+      const int et = threadIdx.x - 64;                // 0..255
+      for (int job = blockIdx.x; job < F.njobs; job += gridDim.x) {
+        const bool idx_stream = job < F.B;
+        const int b = idx_stream ? job : job - F.B;
+        const CompressParams& CP = F.L.p[idx_stream ? 1 : 0];
+        if (CP.d == 512) compress_decode_body<4, 512>(CP, b, part, red, et, 5, 6);
+        else compress_decode_body<4, 128>(CP, b, part, red, et, 5, 6);
+        named_bar_sync(7, 256);   // the job's writes are issued and its shared partials read
+        if (idx_stream && et == 0) {
+          __threadfence();
+          atomicExch(&F.flags[b], 1u);
+        }
+      }
+    }
     const int grp = (warp - 2) >> 2;
     const int gt = threadIdx.x - 64 - 128 * grp;      // 0..127 within the group
     const int quad = warp & 3;                        // TMEM lanes 32*quad .. 32*quad+31
@@ -338,21 +386,22 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
   timeline_mark(status, kTlIndexer, kTlExit);
 }
 
-size_t indexer_smem_bytes(int stages, int N) {
-  return 1024 + (size_t)stages * 32768 + 2 * (size_t)N * 256 + sizeof(IdxSmem) + 2 * 2 * (size_t)N * 4;
+size_t indexer_smem_bytes(int stages, int N, bool fuse) {
+  const size_t base = 1024 + (size_t)stages * 32768 + 2 * (size_t)N * 256 + sizeof(IdxSmem) + 2 * 2 * (size_t)N * 4;
+  return fuse ? base + 16 + kCompressThreads * sizeof(DecodePartial) + kCompressThreads / 32 * sizeof(float) : base;
 }
 
-template __global__ void indexer_kernel<4>(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
-                                           IndexerParams);
-template __global__ void indexer_kernel<8>(const __grid_constant__ CUtensorMap, const __grid_constant__ CUtensorMap,
-                                           IndexerParams);
+template __global__ void indexer_kernel<4>(const __grid_constant__ CUtensorMap,
+                                           const __grid_constant__ CUtensorMap, IndexerParams, IndexerFuse);
+template __global__ void indexer_kernel<8>(const __grid_constant__ CUtensorMap,
+                                           const __grid_constant__ CUtensorMap, IndexerParams, IndexerFuse);
 template __global__ void indexer_kernel<16>(const __grid_constant__ CUtensorMap,
-                                            const __grid_constant__ CUtensorMap, IndexerParams);
+                                           const __grid_constant__ CUtensorMap, IndexerParams, IndexerFuse);
 template __global__ void indexer_kernel<32>(const __grid_constant__ CUtensorMap,
-                                            const __grid_constant__ CUtensorMap, IndexerParams);
+                                           const __grid_constant__ CUtensorMap, IndexerParams, IndexerFuse);
 template __global__ void indexer_kernel<64>(const __grid_constant__ CUtensorMap,
-                                            const __grid_constant__ CUtensorMap, IndexerParams);
+                                           const __grid_constant__ CUtensorMap, IndexerParams, IndexerFuse);
 template __global__ void indexer_kernel<128>(const __grid_constant__ CUtensorMap,
-                                             const __grid_constant__ CUtensorMap, IndexerParams);
+                                           const __grid_constant__ CUtensorMap, IndexerParams, IndexerFuse);
 
 }  // namespace csa

@@ -71,9 +71,20 @@ struct IndexerParams {
   uint32_t* status;
 };
 
+// The decode step's compression, run by the indexer (csa_decode_fused): the epilogue warps of CTA c
+// take jobs c, c + gridDim.x, ... before their first tile. Job j < B compresses request j's index
+// stream (L.p[1]) and then raises flags[j]; job B + j request j's main stream (L.p[0]). The producer
+// waits for flags[b] before it loads the tile holding request b's last visible entry (the one the
+// step may complete) and clears it. njobs = 0: no compression.
+struct IndexerFuse {
+  int njobs, B;
+  uint32_t* flags;                        // [B]; zero between calls
+  CompressLaunch L;
+};
+
 template <int HI>
 __global__ void indexer_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
-                               IndexerParams P);
+                               IndexerParams P, IndexerFuse F);
 
 // ------------------------------------------------------------------------------ top-k (K3)
 
@@ -101,7 +112,7 @@ __global__ void topk_merge_kernel(TopkParams P);
 
 // ------------------------------------------------------------------------------ attention (K4/K5)
 
-constexpr int kAttnThreads = 480;         // warps 0..3 gathers, 4-5 score MMAs, 6 PV MMAs, 7..10 senders, 11..14 softmax
+constexpr int kAttnThreads = 608;         // warps 0..3 gathers, 4-5 score MMAs, 6 PV MMAs, 7..10 senders, 11..18 softmax
 constexpr int kAttnMaxWindow = 1024;
 constexpr int kAttnMaxTopk = 2048;
 constexpr int kAttnMaxCompressed = 2048;  // HCA: visible entries read per query
@@ -178,6 +189,6 @@ int check_indexer_topk_args(int B, int S, int H_I, int d_I, int ratio, int topk,
 
 size_t attn_smem_bytes();
 size_t gemm_smem_bytes();
-size_t indexer_smem_bytes(int stages, int N);
+size_t indexer_smem_bytes(int stages, int N, bool fuse);
 
 }  // namespace csa

@@ -252,7 +252,13 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src) 
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Arrive on `bar` (without raising its expected count) once every cp.async this thread issued so far
+// has landed; the thread does not wait.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Commit this thread's pending cp.async ops and wait until all of them have landed.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // Wait until at most N of this thread's committed cp.async groups are still in flight.
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
