@@ -65,15 +65,22 @@ def test_bindings_refuse_host_tensors():
 
 
 def test_decode_bytes_ledger():
-    """The bench's bytes per decode query: attention reads 1152 rows of 1 KB plus q and output, the
-    indexer the visible index entries plus q_idx, w and the score row."""
+    """The bench's bytes per decode query: attention reads 1152 rows of 1 KB plus q and output; the
+    indexer launch the visible index entries plus q_idx, w and the score row, plus the compressor
+    step it runs (both streams' states and token rows, the entries and the window row)."""
     wl = WORKLOADS["pro_csa_decode_32k"]
     per_q, reads = bench.decode_bytes(wl)
     assert reads == O.reads_per_query(wl.ctx - 1, wl.W, wl.ratio, wl.topk) == 1152
     assert per_q["attention"] == reads * wl.d * 2 + 2 * wl.H * wl.d * 2 + wl.topk * 4
     E = wl.max_entries
-    assert per_q["indexer"] == E * wl.d_I * 2 + wl.H_I * wl.d_I * 2 + wl.H_I * 4 + E * 4
+    comp_main = 2 * 8 * 1024 * 2 + 2 * 1024 * 2 + 512 * 2 + 2 * 512 * 2
+    comp_idx = 2 * 8 * 2 * 128 * 2 + 2 * 2 * 128 * 2 + 128 * 2
+    assert per_q["compress"] == 0
+    assert per_q["indexer"] == E * wl.d_I * 2 + wl.H_I * wl.d_I * 2 + wl.H_I * 4 + E * 4 + comp_main + comp_idx
     assert math.isclose(per_q["attention"] / 1e6, 1.44, rel_tol=0.01)
+    # HCA keeps the compressor launch of its own.
+    per_h, _ = bench.decode_bytes(WORKLOADS["pro_hca_decode_32k"])
+    assert per_h["compress"] > 0 and "indexer" not in per_h
 
 
 def test_graph_rounds_fit_the_timed_steps():
