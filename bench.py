@@ -110,9 +110,10 @@ class ClockSampler:
             pass
 
     def poll_until(self, event, period_s: float = 0.001):
+        self.sample()
         while not event.query():
-            self.sample()
             time.sleep(period_s)
+            self.sample()
 
     def result(self):
         if not self.rows:
@@ -229,6 +230,9 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
         preps[i % len(preps)].launch(stage_events=evs)
 
     nstage = 5 if csa else 3
+    # NVML is opened before the warm-up: its start-up (tens of ms) must not leave the GPU idle, and
+    # its clocks low, just before the timed region.
+    clocks = ClockSampler(torch.cuda.current_device())
     for i in range(args.warmup):
         call(i)
     torch.cuda.synchronize()
@@ -251,26 +255,28 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
             for i in range(per_graph):
                 call(i % len(preps))
         torch.cuda.synchronize()
-        for _ in range(max(1, args.warmup // per_graph)):
+        # Warm replays right before the timed region (at least 2, and at least `warmup` steps), so the
+        # timed steps start on a busy GPU at its running clocks.
+        for _ in range(max(2, -(-args.warmup // per_graph))):
             graph.replay()
-        torch.cuda.synchronize()
+    else:
+        for i in range(args.warmup):
+            call(i)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(torch.cuda.current_device())
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
+    # Every timed step is enqueued before the first clock sample: an NVML query takes milliseconds
+    # of host time, and one taken between launches would leave the device idle inside the timed
+    # region. The samples are taken while the queued steps drain.
     t0.record()
     k = 0
     if graph is not None:
         while k + per_graph <= args.steps:
             graph.replay()
             k += per_graph
-            if (k // per_graph) % max(1, 4 // reps) == 0:
-                clocks.sample()
     for kk in range(k, args.steps):
         call(kk)
-        if kk % 16 == 0:
-            clocks.sample()
     t1.record()
     clocks.poll_until(t1)
     torch.cuda.synchronize()
