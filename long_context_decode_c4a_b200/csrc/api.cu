@@ -228,6 +228,11 @@ int check_compress_args(const csa_compressor_cfg* cfg, int B, int S, const int32
 
 int launch_compress(const CompressLaunch& L, int nstreams, int B, int S, int ratio, cudaStream_t st) {
   if (S == 1) {
+    if (ratio == 128 && nstreams == 1 && L.p[0].d == 512 && L.p[0].overlap == 0) {
+      // C128A with d = 512: a cluster of channel-block CTAs per request.
+      CSA_CUDA(launch_pdl(compress_decode_c128_kernel, dim3(kC128Split, (unsigned)B), dim3(kCompressThreads), 0, st, L));
+      return CSA_OK;
+    }
     CSA_CUDA(launch_pdl(compress_decode_kernel, dim3((unsigned)B, (unsigned)nstreams), dim3(kCompressThreads), 0, st, L));
     return CSA_OK;
   }
@@ -401,7 +406,23 @@ struct AttnArgs {
   int out_is_f32;
   void* ws;
   size_t ws_bytes;
+  size_t part_off = kStatusBytes;  // workspace offset of the split-candidate partials
 };
+
+// Split-candidate attention: a query's candidate tiles are spread over `splits` CTA pairs when the
+// queries alone would leave most SMs idle. The workspace is sized for kAttnSplitPairs pairs (the
+// B200's 148 SMs); a launch uses no more splits than its device's pairs and its workspace allow.
+constexpr int kAttnSplitPairs = 74;
+
+int attn_ws_splits(long long queries) {
+  if (queries <= 0) return 1;
+  return (int)std::max<long long>(1, std::min<long long>(kAttnMaxSplits, kAttnSplitPairs / queries));
+}
+
+size_t attn_part_bytes(long long queries, int splits) {
+  if (splits <= 1) return 0;
+  return (size_t)queries * splits * (128 * 512 + 2 * 128) * sizeof(float);
+}
 
 int check_attn_args(const AttnArgs& a, bool csa_mode) {
   CSA_CHECK_ARG(a.B > 0 && a.S > 0, "B and S must be positive");
@@ -466,7 +487,37 @@ int run_attn(const AttnArgs& a, bool csa_mode, cudaStream_t st) {
   const size_t smem = attn_smem_bytes();
   CSA_CHECK_SUP(smem <= (size_t)dev->max_smem, "shared memory too small for the attention kernel");
   CSA_CHECK_SUP(queries <= 65535, "at most 65535 queries per call");
-  CSA_CUDA(launch_pdl(attn_kernel, dim3(2, (unsigned)queries), dim3(kAttnThreads), smem, st, map_q, P));
+  // Splits: as many as the device's CTA pairs allow per query (and the workspace was sized for),
+  // with at least two tiles of the longest candidate list per split.
+  const long long max_cands = (long long)a.window + (csa_mode ? a.topk : std::min(a.max_entries, kAttnMaxCompressed));
+  const int max_tiles = (int)((max_cands + 31) / 32);
+  int splits = std::min<long long>(attn_ws_splits(queries), std::max<long long>(1, (dev->sms / 2) / queries));
+  splits = std::max(1, std::min(splits, max_tiles / 2));
+  const size_t part_off = round_up(a.part_off, 256);
+  if (splits > 1 && a.ws_bytes < part_off + attn_part_bytes(queries, splits)) splits = 1;
+  P.splits = splits;
+  if (splits > 1) {
+    P.part_o = reinterpret_cast<float*>(static_cast<char*>(a.ws) + part_off);
+    P.part_ml = P.part_o + (size_t)queries * splits * 128 * 512;
+  }
+  CSA_CHECK_SUP(queries * splits <= 65535, "at most 65535 (query, split) items per call");
+  CSA_CUDA(launch_pdl(attn_kernel, dim3(2, (unsigned)(queries * splits)), dim3(kAttnThreads), smem, st, map_q, P));
+  if (splits > 1) {
+    AttnCombineParams C{};
+    C.splits = splits;
+    C.H = a.H;
+    C.d = a.d;
+    C.rope_dim = a.rope_dim;
+    for (int i = 0; i < a.rope_dim / 2; ++i) C.inv_freq[i] = P.inv_freq[i];
+    C.q_pos = a.q_pos;
+    C.part_o = P.part_o;
+    C.part_ml = P.part_ml;
+    C.out = a.out;
+    C.out_is_f32 = P.out_is_f32;
+    C.status = P.status;
+    CSA_CUDA(launch_pdl(attn_combine_kernel, dim3((unsigned)a.H, (unsigned)queries), dim3(kAttnCombineThreads), 0, st,
+                        C));
+  }
   return CSA_OK;
 }
 
@@ -535,13 +586,22 @@ int csa_workspace_size(int kind, int B, int S, int max_entries, int topk, size_t
   CSA_CHECK_ARG(B > 0 && S > 0 && max_entries > 0, "B, S and max_entries must be positive");
   switch (kind) {
     case CSA_WS_INDEXER_TOPK:
-    case CSA_WS_DECODE_FUSED:
       CSA_CHECK_ARG(topk > 0, "topk must be positive");
-      *bytes = indexer_ws_layout((long long)B * S, max_entries, topk, kind == CSA_WS_DECODE_FUSED).total;
+      *bytes = indexer_ws_layout((long long)B * S, max_entries, topk).total;
       return CSA_OK;
+    case CSA_WS_DECODE_FUSED: {
+      CSA_CHECK_ARG(topk > 0, "topk must be positive");
+      const long long q = (long long)B * S;
+      *bytes = indexer_ws_layout(q, max_entries, topk, true).total + attn_part_bytes(q, attn_ws_splits(q));
+      return CSA_OK;
+    }
     case CSA_WS_SPARSE_ATTN:
     case CSA_WS_HCA_ATTN:
-    case CSA_WS_HCA_DECODE_FUSED:
+    case CSA_WS_HCA_DECODE_FUSED: {
+      const long long q = (long long)B * S;
+      *bytes = kStatusBytes + attn_part_bytes(q, attn_ws_splits(q));
+      return CSA_OK;
+    }
     case CSA_WS_OUTPUT_PROJ:
     case CSA_WS_Q_PROJ:
       *bytes = kStatusBytes;
@@ -816,6 +876,7 @@ int csa_decode_fused(const csa_decode_args* a, void* stream) {
   if (int rc = check_attn_args(aa, true)) return rc;
   const IdxWs L = indexer_ws_layout(a->B, a->max_entries, a->topk, true);
   if (int rc = check_ws(a->ws, a->ws_bytes, L.total)) return rc;
+  aa.part_off = L.total;  // the attention's split partials follow the indexer's buffers
 
   uint32_t* status = static_cast<uint32_t*>(a->ws);
   CompressLaunch CL{};

@@ -103,7 +103,8 @@ struct AttnSmem {
   uint64_t drain[3];
   uint32_t tmem_base;
   int abort_flag;
-  int n_tiles;
+  int n_tiles;                        // tiles this CTA pair processes
+  int tile0;                          // the first of them in the query's candidate list
   int bad;
   int epi_bad;                        // some epilogue warp lacks a complete O
   uint32_t scan[kProducers / 32];
@@ -208,6 +209,26 @@ __device__ __forceinline__ void finish_rows(const AttnParams& P, const AttnSmem&
   }
 }
 
+// Split-candidate mode: this CTA's O[:, half] columns [c0, c0 + 32 nchunks) of row h, unnormalised,
+// to the partial buffer row `prow` (fp32). Warp-collective (TMEM loads).
+__device__ __forceinline__ void store_partial_rows(const AttnParams& P, uint32_t o_taddr, int c0, int nchunks,
+                                                   int half, long long prow, int h) {
+#pragma unroll 1
+  for (int cc = 0; cc < nchunks; ++cc) {
+    const int lc = c0 + 32 * cc;
+    uint32_t o[32];
+    tmem_ld32(o_taddr + lc, o);
+    tmem_wait_ld();
+    if (h < P.H) {
+      float4* dst = reinterpret_cast<float4*>(P.part_o + prow * P.d + 256 * half + lc);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        dst[c] = make_float4(__uint_as_float(o[4 * c]), __uint_as_float(o[4 * c + 1]), __uint_as_float(o[4 * c + 2]),
+                             __uint_as_float(o[4 * c + 3]));
+    }
+  }
+}
+
 }  // namespace
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
@@ -225,7 +246,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   const uint32_t half = cluster_ctarank();    // which 256 dims this CTA owns
   const uint32_t peer = half ^ 1u;
   const int nq = P.B * P.S;
-  const int qi = nq - 1 - (int)blockIdx.y;    // later queries (more candidates) first
+  const int item = nq * P.splits - 1 - (int)blockIdx.y;  // later queries (more candidates) first
+  const int qi = item / P.splits;
+  const int sp = item % P.splits;             // which run of the query's tiles (split-candidate mode)
   const int b = qi / P.S;
   volatile int* abort_flag = &sm.abort_flag;
   uint32_t* status = P.status;
@@ -300,6 +323,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     // covers the 512 contiguous bytes of one row per instruction.
     const char* ring_base = reinterpret_cast<const char*>(P.ring) + 512 * half;
     const char* cache_base = reinterpret_cast<const char*>(P.cache) + 512 * half;
+    int tile0 = 0;  // local tile `tile` is tile tile0 + tile of the query's list
     auto issue = [&](int tile) {
       const uint32_t st = smem_u32(stage0 + (size_t)(tile % kStages) * kStageBytes);
 #pragma unroll
@@ -307,16 +331,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         const int c = pt + kProducers * i;  // chunk of the tile
         const int r = c >> 5;               // candidate row 0..31
         const int w = c & 31;               // chunk within the half-row
-        const uint32_t e = sm.list[tile * kTile + r];
+        const uint32_t e = sm.list[(tile0 + tile) * kTile + r];
         const char* src = ((e & kFromCache) ? cache_base : ring_base) + (size_t)(e & kRowMask) * 1024 + w * 16;
         cp_async_16(st + (w >> 3) * kBlockBytes + sw128_offset(r, w & 7), src);
       }
       cp_async_arrive_noinc(&sm.kv_full[tile % kStages]);
     };
     // Tiles made only of window rows are known now: their gathers start before the compressed
-    // entries are read.
+    // entries are read (one pair per query: its tiles start at the window).
     named_bar_sync(2, kProducers);
-    const int w_tiles = min(nwin / kTile, kStages);
+    const int w_tiles = P.splits == 1 ? min(nwin / kTile, kStages) : 0;
     for (int tile = 0; tile < w_tiles; ++tile) issue(tile);
     const int ecap = min((t + 1) / P.ratio, P.max_entries);
     int n = nwin;
@@ -357,13 +381,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     if (bad) sm.bad = 1;
     const int nt = (n + kTile - 1) & ~(kTile - 1);
     for (int k = n + pt; k < nt; k += kProducers) sm.list[k] = self_slot | kInvalid;
-    const int J = nt / kTile;
+    const int Jq = nt / kTile;  // the query's tiles
     // Entries [0, n) are valid, [n, nt) padding.
-    for (int j = pt; j < J; j += kProducers) {
+    for (int j = pt; j < Jq; j += kProducers) {
       const int rem = n - j * kTile;
       sm.mask[j] = rem >= kTile ? 0xFFFFFFFFu : (rem > 0 ? (1u << rem) - 1u : 0u);
     }
-    if (pt == 0) sm.n_tiles = J;
+    // This pair's run of them: tiles [Jq*sp/splits, Jq*(sp+1)/splits).
+    tile0 = (int)(((long long)Jq * sp) / P.splits);
+    const int J = (int)(((long long)Jq * (sp + 1)) / P.splits) - tile0;
+    if (pt == 0) {
+      sm.n_tiles = J;
+      sm.tile0 = tile0;
+    }
     named_bar_sync(2, kProducers);
     if (pt == 0) {
       if (sm.bad && half == 0) record_status(status, CSA_DEV_BOUNDS);
@@ -543,8 +573,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         }
       const float sl = (h < P.H) ? P.sink[h] * 1.4426950408889634f : 0.f;
       float m_used = sl;         // running max in log2 units (starts at the sink), as this group last saw it
-      float l = softB ? 0.f : 1.f;  // this group's part of the denominator, relative to m_used; group 0
-                                 // holds the sink's exp2(sl - m_used) = 1
+      float l = (softB || sp > 0) ? 0.f : 1.f;  // this group's part of the denominator, relative to m_used;
+                                 // group 0 of the first (or only) split holds the sink's exp2(sl - m_used) = 1
+      const int tile0 = sm.tile0;
       // p_free[i % 2] completes once per PV(i): p_free[g] counts the PVs of group g's tiles. A parity
       // wait for PV(i) is unambiguous while the barrier's previous phase (PV(i - 2)) has completed and
       // its next one (PV(i + 2)) cannot have. Each group therefore waits only for: PV(j - 2) of its
@@ -575,7 +606,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         // S = S_0 + S_1 (the same sum in both CTAs), scaled to log2 units; padding -> -inf.
         const uint8_t* xi = xin + c * kXBytes;
         const uint8_t* xm = xout + c * kXBytes;
-        const uint32_t mk = sm.mask[j];
+        const uint32_t mk = sm.mask[tile0 + j];
         float x[32];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -711,12 +742,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
         const int last0 = ((J - 1) & ~1);
         if (done && J > 0 && (!wait_pv(last0) || !wait_pv(J - 1))) done = false;
         if (done && !__all_sync(0xffffffffu, mbar_wait(&sm.b_done, 0, abort_flag, status, 132))) done = false;
+        float m_fin = m_used;
         if (done) {
           const float lb = sm.l_b[h], mb = sm.m_b[h];
-          const float mf = fmaxf(m_used, mb);  // the last published max (it only grows)
+          const float mf = fmaxf(m_used, mb);  // the last published max (it only grows): O's reference
           l = (l != 0.f ? l * exp2f(m_used - mf) : 0.f) + (lb != 0.f ? lb * exp2f(mb - mf) : 0.f);
+          m_fin = mf;
         }
         sm.inv_l[h] = 1.f / l;
+        if (P.splits > 1 && half == 0 && h < P.H) {
+          const long long r = (long long)item * 2 * P.H + h;
+          P.part_ml[r] = m_fin;
+          P.part_ml[r + P.H] = l;
+        }
         j = done ? J : -1;
       }
     }
@@ -734,10 +772,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     uint8_t* srow = stage0 + (size_t)h * kOutRow;  // every gather and MMA reading the stages completed
     if (fin) {
       tc_fence_after();
-      finish_rows(P, sm, tmem + lane_addr + 256, sender ? 128 : 0, 4, (int)half, (long long)qi * P.H + h, h,
-                  sm.inv_l[h], srow);
+      if (P.splits > 1)
+        store_partial_rows(P, tmem + lane_addr + 256, sender ? 128 : 0, 4, (int)half, (long long)item * P.H + h, h);
+      else
+        finish_rows(P, sm, tmem + lane_addr + 256, sender ? 128 : 0, 4, (int)half, (long long)qi * P.H + h, h,
+                    sm.inv_l[h], srow);
+    } else if (P.splits > 1 && J == 0 && j == 0 && h < P.H) {
+      // A split whose run of tiles is empty (the query has fewer tiles than splits): O = 0; its max
+      // and denominator (the sink's term for split 0, nothing otherwise) were stored above.
+      float4* dst = reinterpret_cast<float4*>(P.part_o + ((long long)item * P.H + h) * P.d + 256 * half + (sender ? 128 : 0));
+#pragma unroll 4
+      for (int c = 0; c < 32; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (!P.out_is_f32) {
+    if (!P.out_is_f32 && P.splits == 1) {
       // bf16: each head row's 512 bytes leave in one bulk store, once both roles staged their halves.
       fence_proxy_async_smem();
       named_bar_sync(1, kRoleThreads + kRoleThreads);
@@ -756,6 +803,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) trace_time(status, 255);
   if (warp == kPvWarp) tmem_dealloc(tmem, 512);
   timeline_mark(P.status, kTlAttn, kTlExit);
+}
+
+// Merge of the split-candidate partials of one (query, head) row: with M = max_s m_s and
+// w_s = 2^(m_s - M), o = sum_s w_s O_s / sum_s w_s l_s (the sink is in l_0), then the inverse RoPE
+// of the last rope_dim dims at position t. grid (H, queries); thread i owns dims [4i, 4i + 4).
+__global__ void __launch_bounds__(kAttnCombineThreads) attn_combine_kernel(AttnCombineParams P) {
+  timeline_mark(P.status, kTlCombine, kTlEntry);
+  pdl_wait();
+  pdl_trigger();
+  timeline_mark(P.status, kTlCombine, kTlReady);
+  const int h = blockIdx.x, qi = blockIdx.y, dim = 4 * threadIdx.x;
+  const int ns = P.splits;
+  const long long item0 = (long long)qi * ns;
+  float M = -CUDART_INF_F;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, P.part_ml[(item0 + s) * 2 * P.H + h]);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < ns; ++s) {
+    const long long r = (item0 + s) * 2 * P.H + h;
+    const float ms = P.part_ml[r], ls = P.part_ml[r + P.H];
+    const float w = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
+    L += w * ls;
+    const float4 o = *reinterpret_cast<const float4*>(P.part_o + ((item0 + s) * P.H + h) * P.d + dim);
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  const float inv = 1.f / L;
+  float y[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+  const int rope0 = P.d - P.rope_dim;
+  if (dim >= rope0) {
+    const int t = P.q_pos[qi];
+#pragma unroll
+    for (int c = 0; c < 4; c += 2) {
+      float cs, sn;
+      rope_cos_sin(t, P.inv_freq[(dim + c - rope0) >> 1], &cs, &sn);
+      const float e = y[c], od = y[c + 1];
+      y[c] = e * cs + od * sn;   // rotation by -t
+      y[c + 1] = od * cs - e * sn;
+    }
+  }
+  const long long orow = (long long)qi * P.H + h;
+  if (P.out_is_f32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(P.out) + orow * P.d + dim) = make_float4(y[0], y[1], y[2], y[3]);
+  } else {
+    *reinterpret_cast<uint2*>(static_cast<uint16_t*>(P.out) + orow * P.d + dim) =
+        make_uint2(pack_bf16(y[0], y[1]), pack_bf16(y[2], y[3]));
+  }
+  timeline_mark(P.status, kTlCombine, kTlExit);
 }
 
 size_t attn_smem_bytes() { return 1024 + kStages * kStageBytes + 2 * kXBufs * (size_t)kXBytes + sizeof(AttnSmem); }

@@ -289,6 +289,159 @@ __global__ void __launch_bounds__(kCompressThreads) compress_decode_kernel(Compr
   timeline_mark(P.status, kTlCompress, kTlExit);
 }
 
+// C128A decode step over a cluster of kC128Split CTAs per request (grid: (kC128Split, B)); CTA r of
+// the cluster owns channels [r*CH, r*CH + CH) of the d = 512 (CH = 64). Warp w owns 8 of them and
+// lane l the slots l, l+32, l+64, l+96 of the group: 32 KB of state per CTA read in one round of
+// loads, per-lane partial softmaxes merged across the warp by shuffles. The RMS over all d channels
+// adds the CTAs' partial sums of squares through distributed shared memory. Token t's row (and the
+// window row) go out as 16-byte slices; when t completes its group the state rows read are rows
+// 0..126 (row 127 is token t's own row, taken from the input), so no write aliases a read.
+__global__ void __cluster_dims__(kC128Split, 1, 1) __launch_bounds__(kCompressThreads)
+    compress_decode_c128_kernel(CompressLaunch L) {
+  constexpr int D = 512, RATIO = 128, CH = D / kC128Split, kSlotsPerLane = RATIO / 32;
+  static_assert(CH == 8 * (kCompressThreads / 32), "one warp per 8 channels");
+  __shared__ float red[kCompressThreads / 32];
+  __shared__ float ss_cta;
+  const CompressParams& P = L.p[0];
+  timeline_mark(P.status, kTlCompress, kTlEntry);
+  pdl_wait();
+  pdl_trigger();
+  timeline_mark(P.status, kTlCompress, kTlReady);
+  const int b = blockIdx.y;                      // the same for every CTA of the cluster
+  const int rank = (int)cluster_ctarank();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = P.start_pos[b];
+  if (t < 0) {
+    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    return;                                      // uniform over the cluster: no cluster barrier is skipped alone
+  }
+  const int g = t / RATIO;
+  const int cur = t % RATIO;
+  const bool done = cur == RATIO - 1;
+  uint16_t* skv = P.state_kv + (size_t)b * RATIO * D;
+  uint16_t* ssc = P.state_score + (size_t)b * RATIO * D;
+  const uint16_t* xkv = P.kv + (size_t)b * D;
+  const uint16_t* xsc = P.score + (size_t)b * D;
+  const int ch0 = rank * CH;
+  // Token t's row into state row `cur`, the window row into the ring: 16-byte slices of this CTA's
+  // channels (threads 0-7, 8-15 and 16-23).
+  if (threadIdx.x < 3 * (CH / 8)) {
+    const int part = threadIdx.x / (CH / 8), k = ch0 + 8 * (threadIdx.x % (CH / 8));
+    if (part == 0) {
+      *reinterpret_cast<uint4*>(skv + (size_t)cur * D + k) = *reinterpret_cast<const uint4*>(xkv + k);
+    } else if (part == 1) {
+      *reinterpret_cast<uint4*>(ssc + (size_t)cur * D + k) = *reinterpret_cast<const uint4*>(xsc + k);
+    } else if (P.win_src != nullptr) {
+      uint16_t* dst = P.ring + (long long)b * P.ring_bstride + (long long)(t % P.ring_cap) * D;
+      *reinterpret_cast<uint4*>(dst + k) = *reinterpret_cast<const uint4*>(P.win_src + (size_t)b * D + k);
+    }
+  }
+  if (!done) return;                             // uniform over the cluster
+  if (g >= P.max_entries) {
+    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    return;
+  }
+  const int c0 = ch0 + 8 * w;                    // this warp's 8 channels
+  uint4 kr[kSlotsPerLane], sr[kSlotsPerLane];
+#pragma unroll
+  for (int k = 0; k < kSlotsPerLane; ++k) {
+    const int j = lane + 32 * k;
+    const uint16_t* rk = j == RATIO - 1 ? xkv : skv + (size_t)j * D;
+    const uint16_t* rs = j == RATIO - 1 ? xsc : ssc + (size_t)j * D;
+    kr[k] = *reinterpret_cast<const uint4*>(rk + c0);
+    sr[k] = *reinterpret_cast<const uint4*>(rs + c0);
+  }
+  // Per-channel softmax over the lane's slots in the log2 domain: max m, sum s, weighted sum a.
+  float m[8], s[8], a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    m[i] = -CUDART_INF_F;
+    s[i] = 0.f;
+    a[i] = 0.f;
+  }
+#pragma unroll
+  for (int k = 0; k < kSlotsPerLane; ++k) {
+    const Vec8 kv = load8_regs(kr[k]);
+    const Vec8 sc = load8_regs(sr[k]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float x = sc.v[i] * 1.4426950408889634f;
+      if (x > m[i]) {
+        const float f = exp2f(m[i] - x);
+        s[i] *= f;
+        a[i] *= f;
+        m[i] = x;
+      }
+      const float e = exp2f(x - m[i]);
+      s[i] += e;
+      a[i] += e * kv.v[i];
+    }
+  }
+  // Merge the 32 lanes' partials (butterfly: every lane ends with the whole group's softmax).
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m[i], o);
+      const float s2 = __shfl_xor_sync(0xffffffffu, s[i], o);
+      const float a2 = __shfl_xor_sync(0xffffffffu, a[i], o);
+      const float M = fmaxf(m[i], m2);
+      const float f1 = m[i] == -CUDART_INF_F ? 0.f : exp2f(m[i] - M);
+      const float f2 = m2 == -CUDART_INF_F ? 0.f : exp2f(m2 - M);
+      s[i] = s[i] * f1 + s2 * f2;
+      a[i] = a[i] * f1 + a2 * f2;
+      m[i] = M;
+    }
+  }
+  float x[8], ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[i] = a[i] / s[i];
+    ss += x[i] * x[i];
+  }
+  if (lane == 0) red[w] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < kCompressThreads / 32; ++i) v += red[i];
+    ss_cta = v;
+  }
+  // Every CTA's partial sum of squares is in its shared memory before any CTA reads them.
+  cluster_sync();
+  float tot = 0.f;
+#pragma unroll
+  for (int r = 0; r < kC128Split; ++r) tot += ld_cluster_f32(mapa_shared(smem_u32(&ss_cta), (uint32_t)r));
+  // No CTA leaves (and frees the shared memory the others read) before every read above is done.
+  cluster_sync();
+  if (lane != 0) return;
+  const float rsn = rsqrtf(tot / (float)D + P.eps);
+  const Vec8 gm = load8(P.gamma + c0);
+  float y[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) y[i] = x[i] * rsn * gm.v[i];
+  const int rope0 = D - P.rope_dim;
+  if (c0 >= rope0) {
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+      float cs, sn;
+      rope_cos_sin((long long)g * RATIO, P.inv_freq[(c0 + i - rope0) >> 1], &cs, &sn);
+      const float e = y[i], od = y[i + 1];
+      y[i] = e * cs - od * sn;
+      y[i + 1] = e * sn + od * cs;
+    }
+  }
+  uint16_t* dst = P.cache + (long long)b * P.cache_bstride + (long long)g * D + c0;
+  *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                                              pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+  if (P.cache_f32 != nullptr) {
+    float* df = P.cache_f32 + (long long)b * P.cache_bstride + (long long)g * D + c0;
+    reinterpret_cast<float4*>(df)[0] = make_float4(y[0], y[1], y[2], y[3]);
+    reinterpret_cast<float4*>(df)[1] = make_float4(y[4], y[5], y[6], y[7]);
+  }
+  timeline_mark(P.status, kTlCompress, kTlExit);
+}
+
 // Final state of a multi-token segment: one CTA per request, reads before writes.
 __global__ void __launch_bounds__(kCompressThreads) compress_state_kernel(CompressLaunch L) {
   pdl_wait();

@@ -46,6 +46,8 @@ struct CompressLaunch {
 
 __global__ void compress_kernel(CompressLaunch L);
 __global__ void compress_decode_kernel(CompressLaunch L);
+constexpr int kC128Split = 8;             // CTAs (channel blocks) per request of the C128A decode step
+__global__ void compress_decode_c128_kernel(CompressLaunch L);
 __global__ void compress_state_kernel(CompressLaunch L);
 __global__ void state_reset_kernel(uint16_t* kv, uint16_t* score, long long n);
 
@@ -136,9 +138,32 @@ struct AttnParams {
   void* out;                              // [B*S, H, d]
   int out_is_f32;
   uint32_t* status;
+  // Split-candidate mode (splits > 1): the CTA pair of work item (query qi, split s) takes the s-th
+  // of `splits` contiguous runs of the query's candidate tiles and leaves its unnormalised partial
+  // in part_o [item, H, d] (fp32, O relative to the partial's max) and part_ml [item, 2, H] (the max
+  // in log2 units, then the denominator), item = qi * splits + s; attn_combine_kernel merges them.
+  int splits;
+  float* part_o;
+  float* part_ml;
 };
 
 __global__ void attn_kernel(const __grid_constant__ CUtensorMap map_q, AttnParams P);
+
+constexpr int kAttnMaxSplits = 16;
+constexpr int kAttnCombineThreads = 128;  // one (query, head) row of 512 dims per CTA, 4 per thread
+
+struct AttnCombineParams {
+  int splits, H, d, rope_dim;
+  double inv_freq[kMaxRopePairs];
+  const int32_t* q_pos;
+  const float* part_o;
+  const float* part_ml;
+  void* out;
+  int out_is_f32;
+  uint32_t* status;
+};
+
+__global__ void attn_combine_kernel(AttnCombineParams P);
 
 // ------------------------------------------------------------------------------ output projection
 

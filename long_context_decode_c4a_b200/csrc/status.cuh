@@ -74,7 +74,7 @@ __device__ __forceinline__ void trace_time(uint32_t* status, int idx) {
 // (max) into uint64 words 8 + 3*kernel + {0, 1, 2} of the status area (bytes 64..255 of the
 // workspace, which the caller presets to ~0 / ~0 / 0). Kernel ids: see TimelineKernel. Compiled out
 // otherwise.
-enum TimelineKernel { kTlCompress = 0, kTlIndexer = 1, kTlTopk = 2, kTlTopkMerge = 3, kTlAttn = 4 };
+enum TimelineKernel { kTlCompress = 0, kTlIndexer = 1, kTlTopk = 2, kTlTopkMerge = 3, kTlAttn = 4, kTlCombine = 5 };
 enum TimelineWhat { kTlEntry = 0, kTlReady = 1, kTlExit = 2 };
 __device__ __forceinline__ void timeline_mark(uint32_t* status, int kernel, int what) {
 #ifdef CSA_STEP_TIMELINE

@@ -393,7 +393,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_chunk_kernel(TopkParams P) 
 // lists are in ascending index order and chunk order is index order, so position order in the
 // concatenation is index order (unused slots are marked invalid).
 __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) {
-  __shared__ TopkShared sh;
+  __shared__ TopkRegShared sh;
   __shared__ int cnts[kTopkMaxChunks];
   timeline_mark(P.status, kTlTopkMerge, kTlEntry);
   pdl_wait();
@@ -415,7 +415,32 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) 
   const int K = P.topk;
   auto key_of = [&](int i) -> uint32_t { return (i % K) < cnts[i / K] ? ck[i] : 0u; };
   int32_t* out = P.out + (long long)q * P.topk;
-  const uint32_t cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = ci[i]; }, sh);
+  uint32_t cnt;
+  constexpr int KPT = kTopkChunk / kTopkThreads;
+  if (n <= KPT * kTopkThreads) {
+    // The union fits the registers (16 per thread): the same register-resident select as a chunk.
+    // Thread t holds positions [t*KPT, t*KPT + KPT) of the concatenation.
+    uint32_t key[KPT];
+    const int p0 = (int)threadIdx.x * KPT;
+    if (K % KPT == 0 && p0 + KPT <= n) {
+      // The thread's positions lie in one chunk's list: one count check, vector loads.
+      const int c = p0 / K, s0 = p0 % K;
+      const uint4* src = reinterpret_cast<const uint4*>(ck + p0);
+#pragma unroll
+      for (int v = 0; v < KPT / 4; ++v) {
+        const uint4 u = src[v];
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) key[4 * v + e] = (s0 + 4 * v + e) < cnts[c] ? w4[e] : 0u;
+      }
+    } else {
+#pragma unroll
+      for (int r = 0; r < KPT; ++r) key[r] = p0 + r < n ? key_of(p0 + r) : 0u;
+    }
+    cnt = block_topk_regs<kTopkThreads, KPT>(key, P.topk, [&](uint32_t pos, int r) { out[pos] = ci[p0 + r]; }, sh);
+  } else {
+    cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = ci[i]; }, sh.t);
+  }
   for (int j = cnt + threadIdx.x; j < P.topk; j += blockDim.x) out[j] = -1;
   timeline_mark(P.status, kTlTopkMerge, kTlExit);
 }

@@ -83,7 +83,16 @@ def test_workspace_sizes(lib):
     # long rows need the chunked top-k lists: 16 chunks x 1024 (key, index) pairs per query
     assert n.value >= 256 + 8 * 262144 * 4 + 2 * 8 * 16 * 1024 * 4
     assert lib.csa_workspace_size(_lib.CSA_WS_HCA_ATTN, 64, 1, 256, 0, ctypes.byref(n)) == 0
-    assert n.value == 256
+    assert n.value == 256      # 64 queries: one CTA pair each, no split partials
+    # 8 queries: each query's candidates are split over 74 // 8 = 9 CTA pairs, whose partials
+    # (O: 128 x 512 fp32, max and denominator: 2 x 128 fp32) live in the workspace
+    per_split = (128 * 512 + 2 * 128) * 4
+    assert lib.csa_workspace_size(_lib.CSA_WS_SPARSE_ATTN, 8, 1, 262144, 1024, ctypes.byref(n)) == 0
+    assert n.value == 256 + 8 * 9 * per_split
+    assert lib.csa_workspace_size(_lib.CSA_WS_DECODE_FUSED, 8, 1, 262144, 1024, ctypes.byref(n)) == 0
+    assert n.value >= 256 + 8 * 262144 * 4 + 2 * 8 * 16 * 1024 * 4 + 8 * 9 * per_split
+    assert lib.csa_workspace_size(_lib.CSA_WS_SPARSE_ATTN, 1, 1, 64, 8, ctypes.byref(n)) == 0
+    assert n.value == 256 + 16 * per_split   # at most 16 splits
     assert lib.csa_workspace_size(_lib.CSA_WS_OUTPUT_PROJ, 1, 1, 1, 1, ctypes.byref(n)) == 0
     assert n.value == 256
     assert lib.csa_workspace_size(99, 1, 1, 1, 1, ctypes.byref(n)) == _lib.CSA_ERR_INVALID_ARG

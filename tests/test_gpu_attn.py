@@ -146,7 +146,53 @@ def test_csa_with_all_entries_equals_hca(ops):
         topk[b, 0, :E] = torch.arange(E, dtype=torch.int32)
     o1 = torch.empty(B, S, H, d, dtype=torch.float32, device="cuda")
     o2 = torch.empty_like(o1)
-    ops.sparse_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), topk.cuda(), sink.cuda(), W, out=o1)
-    ops.hca_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), sink.cuda(), W, ratio=4, out=o2)
+    # Status-only workspaces: one CTA pair per query in both calls, so the arithmetic is the same.
+    ws1 = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ws2 = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    ops.sparse_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), topk.cuda(), sink.cuda(), W, out=o1, ws=ws1)
+    ops.hca_attn(pos.cuda(), q.cuda(), ring.cuda(), cache.cuda(), sink.cuda(), W, ratio=4, out=o2, ws=ws2)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("mode", ["csa", "hca"])
+def test_split_candidates_match_one_pair_per_query(ops, mode):
+    """Split-candidate mode (a query's tiles spread over several CTA pairs, partials merged by
+    log-sum-exp) against one pair per query (a status-only workspace) and against the oracle. Query
+    0 sits at t = 0 (one candidate: most splits are empty, split 0 holds the sink), query 3 at a
+    position with a ragged last tile."""
+    g = torch.Generator().manual_seed(21)
+    B, S, H, d, W = 4, 1, 128, 512, 128
+    pos = torch.tensor([[0], [32767], [1500], [4242]], dtype=torch.int32)
+    E_cap = 8192 if mode == "csa" else 256
+    q = _q(B, S, H, d, g)
+    ring = torch.randn(B, W, d, generator=g).to(torch.bfloat16)
+    cache = torch.randn(B, E_cap, d, generator=g).to(torch.bfloat16)
+    sink = torch.randn(H, generator=g)
+    args = [pos.cuda(), q.cuda(), ring.cuda(), cache.cuda()]
+    topk = _random_topk(B, S, pos, 1024, 4, g) if mode == "csa" else None
+    kind = ops._lib.CSA_WS_SPARSE_ATTN if mode == "csa" else ops._lib.CSA_WS_HCA_ATTN
+    ws_split = ops.workspace(kind, B, S, 1, 1, "cuda")
+    assert ws_split.numel() > 256          # the workspace holds the partials of several splits per query
+    outs = []
+    for ws in (ws_split, torch.zeros(256, dtype=torch.uint8, device="cuda")):
+        out = torch.empty(B, S, H, d, dtype=torch.float32, device="cuda")
+        if mode == "csa":
+            ops.sparse_attn(*args, topk.cuda(), sink.cuda(), W, out=out, ws=ws)
+        else:
+            ops.hca_attn(*args, sink.cuda(), W, ratio=128, out=out, ws=ws)
+        torch.cuda.synchronize()
+        assert ops.device_status(ws) == 0
+        outs.append(out)
+    split, single = outs
+    for b in range(B):
+        t = int(pos[b, 0])
+        sel = np64(topk[b, 0]).tolist() if mode == "csa" else list(range(min((t + 1) // 128, E_cap)))
+        ref = O.attend_query(np64(q[b, 0]), t, W, np64(ring[b]), W, np64(cache[b]), sel, np64(sink),
+                             1 / math.sqrt(d), 64, 10000.0)
+        assert_attn_close(split[b, 0], ref, f"{mode} split b={b} t={t}")
+        assert_attn_close(single[b, 0], ref, f"{mode} one pair b={b} t={t}")
+    # The two differ only by rounding (other running maxima for P's bf16 parts, another order of the
+    # same sums): far below what a dropped or misweighted split would leave.
+    rms = single.float().square().mean().sqrt()
+    assert float((split - single).abs().max()) <= 2e-3 * float(rms)
