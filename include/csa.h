@@ -97,6 +97,11 @@ enum {
  * The workspace must be 256-byte aligned. Its first 256 bytes hold the device status word;
  * the caller zeroes the whole workspace once before first use (later calls keep the status
  * word sticky until csa_get_device_status clears it).
+ * The attention kinds (and CSA_WS_DECODE_FUSED) also hold, for small batches (B*S <= 37), the
+ * partial results of split-candidate attention: a query's candidates are then spread over
+ * min(16, 74 / (B*S)) CTA pairs, each leaving 128 x 512 + 2 x 128 floats that a second kernel
+ * merges. A smaller workspace (down to the 256-byte status word) is accepted by the attention
+ * entry points: they then run one CTA pair per query (same results up to rounding, slower).
  */
 CSA_API int csa_workspace_size(int kind, int B, int S, int max_entries, int topk, size_t* bytes);
 
