@@ -233,12 +233,26 @@ __device__ uint32_t block_topk(int n, int k, KeyFn key_of, EmitFn emit, TopkShar
 }
 
 constexpr int kCandCap = 4096;   // keys of the threshold bin after the first pass, kept in smem
+constexpr int kRankMax = 128;    // at most this many: the threshold is found by ranking them directly
 
 struct TopkRegShared {
   TopkShared t;
   uint32_t cand[kCandCap];
   uint32_t ncand;
+  uint32_t T, need;                // threshold found by ranking the candidates
 };
+
+// Exclusive prefix (in thread order) and totals of two per-thread counts below 2^16 each, with
+// one block scan of the packed pair (the totals stay below 2^16: no carry between the halves).
+__device__ __forceinline__ void block_scan2_packed(uint32_t a, uint32_t b, SelectShared& sh, uint32_t& pre_a,
+                                                   uint32_t& pre_b, uint32_t& tot_a, uint32_t& tot_b) {
+  uint32_t tot;
+  const uint32_t pre = block_excl_scan((a << 16) | b, sh, tot);
+  pre_a = pre >> 16;
+  pre_b = pre & 0xFFFFu;
+  tot_a = tot >> 16;
+  tot_b = tot & 0xFFFFu;
+}
 
 // Top-k of up to KPT * blockDim keys held in registers (0 = empty position); thread t holds the
 // keys of positions t*KPT .. t*KPT+KPT-1. The first radix pass runs over the registers; the keys
@@ -261,20 +275,47 @@ __device__ uint32_t block_topk_regs(const uint32_t (&key)[KPT], int k, EmitFn em
     if (lo != hi) {
       if (tid == 0) sh.ncand = 0;
       __syncthreads();
+      // The keys left in [lo, hi] go to shared memory: one counter update per warp.
       const uint32_t lt = (1u << lane) - 1u;
+      uint32_t bal[KPT];
+      uint32_t wcnt = 0;
 #pragma unroll
       for (int r = 0; r < KPT; ++r) {
-        const bool in = key[r] >= lo && key[r] <= hi;
-        const uint32_t m = __ballot_sync(0xffffffffu, in);
-        uint32_t base = 0;
-        if (lane == 0 && m != 0u) base = atomicAdd(&sh.ncand, (uint32_t)__popc(m));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        const uint32_t pos = base + (uint32_t)__popc(m & lt);
-        if (in && pos < (uint32_t)kCandCap) sh.cand[pos] = key[r];
+        bal[r] = __ballot_sync(0xffffffffu, key[r] >= lo && key[r] <= hi);
+        wcnt += (uint32_t)__popc(bal[r]);
+      }
+      uint32_t base = 0;
+      if (lane == 0 && wcnt != 0u) base = atomicAdd(&sh.ncand, wcnt);
+      base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+      for (int r = 0; r < KPT; ++r) {
+        const uint32_t pos = base + (uint32_t)__popc(bal[r] & lt);
+        if (((bal[r] >> lane) & 1u) && pos < (uint32_t)kCandCap) sh.cand[pos] = key[r];
+        base += (uint32_t)__popc(bal[r]);
       }
       __syncthreads();
       const uint32_t nc = sh.ncand;
-      if (nc <= (uint32_t)kCandCap) {
+      if (nc <= (uint32_t)kRankMax) {
+        // Few candidates: the krem-th largest of them is the key c with g < krem <= g + e, where g
+        // (e) counts the candidates greater than (equal to) c; need = krem - g. (Each candidate's
+        // thread reads all nc: worth it only while nc is small.)
+        if (tid < (int)nc) {
+          const uint32_t c = sh.cand[tid];
+          uint32_t g = 0, e = 0;
+          for (uint32_t j = 0; j < nc; ++j) {
+            const uint32_t x = sh.cand[j];
+            g += x > c ? 1u : 0u;
+            e += x == c ? 1u : 0u;
+          }
+          if (g < krem && krem <= g + e) {  // every thread holding T writes the same values
+            sh.T = c;
+            sh.need = krem - g;
+          }
+        }
+        __syncthreads();
+        lo = hi = sh.T;
+        krem = sh.need;
+      } else if (nc <= (uint32_t)kCandCap) {
         auto list = [&](auto&& f) {
           for (uint32_t i = tid; i < nc; i += NT) f(sh.cand[i]);
         };
@@ -294,8 +335,9 @@ __device__ uint32_t block_topk_regs(const uint32_t (&key)[KPT], int k, EmitFn em
     if (take_all || key[r] > T) ++n_gt;
     else if (key[r] == T) ++n_eq;
   }
+  static_assert(KPT * NT < 65536, "packed counts");
   uint32_t pre_gt, pre_eq, tot_gt, tot_eq;
-  block_scan2(n_gt, n_eq, sh.t, pre_gt, pre_eq, tot_gt, tot_eq);
+  block_scan2_packed(n_gt, n_eq, sh.t.sel, pre_gt, pre_eq, tot_gt, tot_eq);
   uint32_t eq_seen = pre_eq;                       // keys == T before this thread's range
   uint32_t pos = pre_gt + min(pre_eq, need);       // output slot of the next chosen key
 #pragma unroll
@@ -421,23 +463,34 @@ __global__ void __launch_bounds__(kTopkThreads) topk_merge_kernel(TopkParams P) 
     // The union fits the registers (16 per thread): the same register-resident select as a chunk.
     // Thread t holds positions [t*KPT, t*KPT + KPT) of the concatenation.
     uint32_t key[KPT];
+    int32_t idx[KPT];
     const int p0 = (int)threadIdx.x * KPT;
     if (K % KPT == 0 && p0 + KPT <= n) {
-      // The thread's positions lie in one chunk's list: one count check, vector loads.
+      // The thread's positions lie in one chunk's list: one count check, vector loads of the keys
+      // and of their indices.
       const int c = p0 / K, s0 = p0 % K;
       const uint4* src = reinterpret_cast<const uint4*>(ck + p0);
+      const int4* isrc = reinterpret_cast<const int4*>(ci + p0);
 #pragma unroll
       for (int v = 0; v < KPT / 4; ++v) {
         const uint4 u = src[v];
+        const int4 iv = isrc[v];
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+        const int32_t i4[4] = {iv.x, iv.y, iv.z, iv.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) key[4 * v + e] = (s0 + 4 * v + e) < cnts[c] ? w4[e] : 0u;
+        for (int e = 0; e < 4; ++e) {
+          key[4 * v + e] = (s0 + 4 * v + e) < cnts[c] ? w4[e] : 0u;
+          idx[4 * v + e] = i4[e];
+        }
       }
     } else {
 #pragma unroll
-      for (int r = 0; r < KPT; ++r) key[r] = p0 + r < n ? key_of(p0 + r) : 0u;
+      for (int r = 0; r < KPT; ++r) {
+        key[r] = p0 + r < n ? key_of(p0 + r) : 0u;
+        idx[r] = key[r] != 0u ? ci[p0 + r] : -1;
+      }
     }
-    cnt = block_topk_regs<kTopkThreads, KPT>(key, P.topk, [&](uint32_t pos, int r) { out[pos] = ci[p0 + r]; }, sh);
+    cnt = block_topk_regs<kTopkThreads, KPT>(key, P.topk, [&](uint32_t pos, int r) { out[pos] = idx[r]; }, sh);
   } else {
     cnt = block_topk(n, P.topk, key_of, [&](uint32_t pos, int i) { out[pos] = ci[i]; }, sh.t);
   }
