@@ -306,8 +306,33 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
                 for i, n in enumerate(stage_names)}
 
     launches_per_step = (4 + (1 if wl.max_entries > 16384 else 0)) if csa else 2
+    # ---- single-step latency: one step per replay of a one-step CUDA graph, the device idle before
+    # it (synchronised between steps), events on the launching stream. This is what one decode step
+    # of this layer costs on its own, without the overlap of consecutive steps' launches.
+    one = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        call(0)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(one):
+        call(0)
+    lat = []
+    for k in range(max(8, min(args.steps, 50)) + 3):
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        one.replay()
+        z.record()
+        torch.cuda.synchronize()
+        if k >= 3:
+            lat.append(a.elapsed_time(z))
+    single_ms = max_over_ranks(statistics.median(lat), world)
+    del one
     if light:
-        return dict(ms=ms, stage_ms=stage_ms, clocks=clk, launches=launches_per_step * args.steps)
+        return dict(ms=ms, stage_ms=stage_ms, clocks=clk, launches=launches_per_step * args.steps,
+                    single_ms=single_ms)
     # ---- end-to-end through the public API with host buffers: every step copies its inputs from
     # pinned host memory, runs, and copies its output back. Copies run on their own streams and
     # overlap the neighbouring steps' compute (two device buffer sets, events between streams).
@@ -370,7 +395,7 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     return dict(ms=ms, stage_ms=stage_ms, clocks=clk, e2e_ms=e2e_ms, h2d=h2d, d2h=d2h,
-                launches=launches_per_step * args.steps)
+                launches=launches_per_step * args.steps, single_ms=single_ms)
 
 
 def prefill_ledger(wl):
@@ -525,7 +550,8 @@ def extra_workloads(args, peaks):
         per_q, reads = decode_bytes(wl)
         total = sum(per_q.values()) * wl.B
         res[name] = {"value": wl.B * 1000.0 / r["ms"], "unit": "queries/s", "tokens_per_s": wl.B * 1000.0 / r["ms"],
-                     "ms_per_step": r["ms"], "kernels_ms": r["stage_ms"], "reads_per_query": reads,
+                     "ms_per_step": r["ms"], "single_step_latency_us": r["single_ms"] * 1e3,
+                     "kernels_ms": r["stage_ms"], "reads_per_query": reads,
                      "roofline": {"bound": "hbm", "achieved": total / (r["ms"] * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
                                   "unit": "GB/s", "frac": total / (r["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
                                   "scope": "whole step, algorithmic bytes"}}
@@ -710,6 +736,9 @@ def main(argv=None):
         "e2e": {"value": B_total * 1000.0 / r["e2e_ms"], "unit": "queries/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"]},
         "gpu_launches": r["launches"],
+        "single_step": {"latency_us": r["single_ms"] * 1e3,
+                        "how": "one step per replay of a one-step CUDA graph, synchronised between steps "
+                               "(no overlap with neighbouring steps); median, CUDA events on the launching stream"},
         "clocks": r["clocks"],
     }
     if world == 1 and not args.no_extra:

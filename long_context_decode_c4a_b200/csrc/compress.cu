@@ -290,18 +290,27 @@ __global__ void __launch_bounds__(kCompressThreads) compress_decode_kernel(Compr
 }
 
 // C128A decode step over a cluster of kC128Split CTAs per request (grid: (kC128Split, B)); CTA r of
-// the cluster owns channels [r*CH, r*CH + CH) of the d = 512 (CH = 64). Warp w owns 8 of them and
-// lane l the slots l, l+32, l+64, l+96 of the group: 32 KB of state per CTA read in one round of
-// loads, per-lane partial softmaxes merged across the warp by shuffles. The RMS over all d channels
-// adds the CTAs' partial sums of squares through distributed shared memory. Token t's row (and the
-// window row) go out as 16-byte slices; when t completes its group the state rows read are rows
-// 0..126 (row 127 is token t's own row, taken from the input), so no write aliases a read.
+// the cluster owns channels [r*CH, r*CH + CH) of the d = 512 (CH = 64, 8 chunks of 8). Thread t
+// takes chunk t % 8 of the slots (t / 8) + 32k, k = 0..3: a warp load covers 128 contiguous bytes
+// of each of 4 slot rows, and the CTA reads its 32 KB of state in one round of loads. The softmax
+// over the 128 slots of each channel: the max over a thread's slots, across the warp (lanes 8
+// apart share the channels) and across the warps (shared memory); then the terms against that max,
+// summed the same way. The RMS over all d channels adds the CTAs' partial sums of squares through
+// distributed shared memory. Token t's row (and the window row) go out as 16-byte slices; when t
+// completes its group the state rows read are rows 0..126 (row 127 is token t's own row, taken
+// from the input), so no write aliases a read.
 __global__ void __cluster_dims__(kC128Split, 1, 1) __launch_bounds__(kCompressThreads)
     compress_decode_c128_kernel(CompressLaunch L) {
-  constexpr int D = 512, RATIO = 128, CH = D / kC128Split, kSlotsPerLane = RATIO / 32;
-  static_assert(CH == 8 * (kCompressThreads / 32), "one warp per 8 channels");
-  __shared__ float red[kCompressThreads / 32];
-  __shared__ float ss_cta;
+  constexpr int D = 512, RATIO = 128, CH = D / kC128Split, NCH = CH / 8;
+  constexpr int kGroups = kCompressThreads / NCH;   // slot groups (32)
+  constexpr int kPer = RATIO / kGroups;             // slots per thread (4)
+  constexpr int kWarps = kCompressThreads / 32;
+  static_assert(NCH == 8 && kGroups == 32 && kPer == 4, "thread layout");
+  __shared__ float red_m[kWarps][CH];   // per-warp partial max, then partial sums of the terms
+  __shared__ float red_a[kWarps][CH];   // per-warp partial weighted sums
+  __shared__ float ch_m[CH];            // the channels' max
+  __shared__ float ss_w[CH / 8];
+  __shared__ float ss_all[kC128Split];  // every CTA's partial sum of squares, written by that CTA
   const CompressParams& P = L.p[0];
   timeline_mark(P.status, kTlCompress, kTlEntry);
   pdl_wait();
@@ -309,10 +318,10 @@ __global__ void __cluster_dims__(kC128Split, 1, 1) __launch_bounds__(kCompressTh
   timeline_mark(P.status, kTlCompress, kTlReady);
   const int b = blockIdx.y;                      // the same for every CTA of the cluster
   const int rank = (int)cluster_ctarank();
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int t = P.start_pos[b];
   if (t < 0) {
-    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    if (tid == 0) record_status(P.status, CSA_DEV_BOUNDS);
     return;                                      // uniform over the cluster: no cluster barrier is skipped alone
   }
   const int g = t / RATIO;
@@ -325,8 +334,8 @@ __global__ void __cluster_dims__(kC128Split, 1, 1) __launch_bounds__(kCompressTh
   const int ch0 = rank * CH;
   // Token t's row into state row `cur`, the window row into the ring: 16-byte slices of this CTA's
   // channels (threads 0-7, 8-15 and 16-23).
-  if (threadIdx.x < 3 * (CH / 8)) {
-    const int part = threadIdx.x / (CH / 8), k = ch0 + 8 * (threadIdx.x % (CH / 8));
+  if (tid < 3 * NCH) {
+    const int part = tid / NCH, k = ch0 + 8 * (tid % NCH);
     if (part == 0) {
       *reinterpret_cast<uint4*>(skv + (size_t)cur * D + k) = *reinterpret_cast<const uint4*>(xkv + k);
     } else if (part == 1) {
@@ -338,106 +347,134 @@ __global__ void __cluster_dims__(kC128Split, 1, 1) __launch_bounds__(kCompressTh
   }
   if (!done) return;                             // uniform over the cluster
   if (g >= P.max_entries) {
-    if (threadIdx.x == 0) record_status(P.status, CSA_DEV_BOUNDS);
+    if (tid == 0) record_status(P.status, CSA_DEV_BOUNDS);
     return;
   }
-  const int c0 = ch0 + 8 * w;                    // this warp's 8 channels
-  uint4 kr[kSlotsPerLane], sr[kSlotsPerLane];
+  const int chunk = tid % NCH, grp = tid / NCH;
+  const int c0 = ch0 + 8 * chunk;                // this thread's 8 channels
+  uint4 kr[kPer], sr[kPer];
 #pragma unroll
-  for (int k = 0; k < kSlotsPerLane; ++k) {
-    const int j = lane + 32 * k;
+  for (int k = 0; k < kPer; ++k) {
+    const int j = grp + kGroups * k;
     const uint16_t* rk = j == RATIO - 1 ? xkv : skv + (size_t)j * D;
     const uint16_t* rs = j == RATIO - 1 ? xsc : ssc + (size_t)j * D;
     kr[k] = *reinterpret_cast<const uint4*>(rk + c0);
     sr[k] = *reinterpret_cast<const uint4*>(rs + c0);
   }
-  // Per-channel softmax over the lane's slots in the log2 domain: max m, sum s, weighted sum a.
-  float m[8], s[8], a[8];
+  // Max over the thread's slots (log2 domain), then over the lanes with the same chunk (xor 8,
+  // 16), then over the warps.
+  Vec8 kv[kPer], sc[kPer];
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = -CUDART_INF_F;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    kv[k] = load8_regs(kr[k]);
+    sc[k] = load8_regs(sr[k]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      sc[k].v[i] *= 1.4426950408889634f;  // log2(e)
+      m[i] = fmaxf(m[i], sc[k].v[i]);
+    }
+  }
+#pragma unroll
+  for (int o = NCH; o < 32; o <<= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], __shfl_xor_sync(0xffffffffu, m[i], o));
+  if (lane < NCH) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red_m[w][8 * chunk + i] = m[i];
+  }
+  __syncthreads();
+  if (tid < CH) {
+    float v = red_m[0][tid];
+#pragma unroll
+    for (int q = 1; q < kWarps; ++q) v = fmaxf(v, red_m[q][tid]);
+    ch_m[tid] = v;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = ch_m[8 * chunk + i];
+  // Terms against the max: their sum s and the weighted sum a, reduced the same way.
+  float s[8], a[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    m[i] = -CUDART_INF_F;
     s[i] = 0.f;
     a[i] = 0.f;
   }
 #pragma unroll
-  for (int k = 0; k < kSlotsPerLane; ++k) {
-    const Vec8 kv = load8_regs(kr[k]);
-    const Vec8 sc = load8_regs(sr[k]);
+  for (int k = 0; k < kPer; ++k)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float x = sc.v[i] * 1.4426950408889634f;
-      if (x > m[i]) {
-        const float f = exp2f(m[i] - x);
-        s[i] *= f;
-        a[i] *= f;
-        m[i] = x;
-      }
-      const float e = exp2f(x - m[i]);
+      const float e = exp2f(sc[k].v[i] - m[i]);
       s[i] += e;
-      a[i] += e * kv.v[i];
+      a[i] += e * kv[k].v[i];
     }
-  }
-  // Merge the 32 lanes' partials (butterfly: every lane ends with the whole group's softmax).
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int o = NCH; o < 32; o <<= 1)
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m[i], o);
-      const float s2 = __shfl_xor_sync(0xffffffffu, s[i], o);
-      const float a2 = __shfl_xor_sync(0xffffffffu, a[i], o);
-      const float M = fmaxf(m[i], m2);
-      const float f1 = m[i] == -CUDART_INF_F ? 0.f : exp2f(m[i] - M);
-      const float f2 = m2 == -CUDART_INF_F ? 0.f : exp2f(m2 - M);
-      s[i] = s[i] * f1 + s2 * f2;
-      a[i] = a[i] * f1 + a2 * f2;
-      m[i] = M;
+      s[i] += __shfl_xor_sync(0xffffffffu, s[i], o);
+      a[i] += __shfl_xor_sync(0xffffffffu, a[i], o);
+    }
+  if (lane < NCH) {  // (every read of the maxima in red_m preceded the last barrier)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      red_m[w][8 * chunk + i] = s[i];
+      red_a[w][8 * chunk + i] = a[i];
     }
   }
-  float x[8], ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    x[i] = a[i] / s[i];
-    ss += x[i] * x[i];
-  }
-  if (lane == 0) red[w] = ss;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  // Thread c < CH finishes channel ch0 + c: x = a / s, and its square for the RMS.
+  float x = 0.f;
+  if (tid < CH) {
+    float S = 0.f, A = 0.f;
+#pragma unroll
+    for (int q = 0; q < kWarps; ++q) {
+      S += red_m[q][tid];
+      A += red_a[q][tid];
+    }
+    x = A / S;
+    float sq = x * x;
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    if ((tid & 7) == 0) ss_w[tid >> 3] = sq;
+  }
+  __syncthreads();
+  if (tid < kC128Split) {
+    // Thread r stores this CTA's partial into slot `rank` of CTA r's ss_all.
     float v = 0.f;
 #pragma unroll
-    for (int i = 0; i < kCompressThreads / 32; ++i) v += red[i];
-    ss_cta = v;
+    for (int i = 0; i < CH / 8; ++i) v += ss_w[i];
+    st_cluster_f32(mapa_shared(smem_u32(&ss_all[rank]), (uint32_t)tid), v);
   }
-  // Every CTA's partial sum of squares is in its shared memory before any CTA reads them.
+  // Every partial has landed in every CTA's shared memory; nothing crosses CTAs after this
+  // barrier, so a CTA may leave as soon as it is done.
   cluster_sync();
+  if (tid >= CH) return;
   float tot = 0.f;
 #pragma unroll
-  for (int r = 0; r < kC128Split; ++r) tot += ld_cluster_f32(mapa_shared(smem_u32(&ss_cta), (uint32_t)r));
-  // No CTA leaves (and frees the shared memory the others read) before every read above is done.
-  cluster_sync();
-  if (lane != 0) return;
-  const float rsn = rsqrtf(tot / (float)D + P.eps);
-  const Vec8 gm = load8(P.gamma + c0);
-  float y[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) y[i] = x[i] * rsn * gm.v[i];
+  for (int r = 0; r < kC128Split; ++r) tot += ss_all[r];
+  // Channel c = ch0 + tid: RMSNorm, gamma, RoPE on the rotated channels (pairs in adjacent threads).
+  const int c = ch0 + tid;
+  const float gm = __uint_as_float((uint32_t)P.gamma[c] << 16);
+  float y = x * rsqrtf(tot / (float)D + P.eps) * gm;
   const int rope0 = D - P.rope_dim;
-  if (c0 >= rope0) {
-#pragma unroll
-    for (int i = 0; i < 8; i += 2) {
-      float cs, sn;
-      rope_cos_sin((long long)g * RATIO, P.inv_freq[(c0 + i - rope0) >> 1], &cs, &sn);
-      const float e = y[i], od = y[i + 1];
-      y[i] = e * cs - od * sn;
-      y[i + 1] = e * sn + od * cs;
-    }
+  const float yo = __shfl_xor_sync(0xffffffffu, y, 1);   // the other element of the pair
+  if (c >= rope0) {
+    float cs, sn;
+    rope_cos_sin((long long)g * RATIO, P.inv_freq[(c - rope0) >> 1], &cs, &sn);
+    y = (c & 1) ? yo * sn + y * cs : y * cs - yo * sn;
   }
-  uint16_t* dst = P.cache + (long long)b * P.cache_bstride + (long long)g * D + c0;
-  *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                                              pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
-  if (P.cache_f32 != nullptr) {
-    float* df = P.cache_f32 + (long long)b * P.cache_bstride + (long long)g * D + c0;
-    reinterpret_cast<float4*>(df)[0] = make_float4(y[0], y[1], y[2], y[3]);
-    reinterpret_cast<float4*>(df)[1] = make_float4(y[4], y[5], y[6], y[7]);
+  // Pack pairs of channels: even threads store 2 bf16 (and 2 fp32).
+  const float y1 = __shfl_xor_sync(0xffffffffu, y, 1);
+  if ((tid & 1) == 0) {
+    uint16_t* dst = P.cache + (long long)b * P.cache_bstride + (long long)g * D + c;
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(y, y1);
+    if (P.cache_f32 != nullptr) {
+      float* df = P.cache_f32 + (long long)b * P.cache_bstride + (long long)g * D + c;
+      *reinterpret_cast<float2*>(df) = make_float2(y, y1);
+    }
   }
   timeline_mark(P.status, kTlCompress, kTlExit);
 }
