@@ -163,6 +163,19 @@ def graph_rounds(requested: int, steps: int, sets: int) -> int:
     return max(1, min(requested, steps // max(1, sets)))
 
 
+def decode_launches(wl) -> int:
+    """Kernels one decode step launches, by the library's rules: CSA = indexer (with the compressor
+    step) + top-k (one launch up to 16384 entries per row, chunks + merge beyond) + attention; HCA =
+    the C128A step + attention; plus the combine kernel when the attention splits each query's
+    candidates over several CTA pairs (at most 16, 74 // queries and half the longest list's tiles)."""
+    cands = wl.W + (wl.topk if wl.has_indexer else min(wl.max_entries, 2048))
+    splits = max(1, min(16, 74 // max(1, wl.B * wl.S), ((cands + 31) // 32) // 2))
+    n = 2 + (1 if splits > 1 else 0)
+    if wl.has_indexer:
+        n += 1 if wl.max_entries <= 16384 else 2
+    return n
+
+
 def decode_bytes(wl):
     """Algorithmic HBM bytes per query of each kernel of one CSA/HCA decode step."""
     E = wl.max_entries
@@ -305,7 +318,7 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
     stage_ms = {n: statistics.mean(stage_ev[k][i].elapsed_time(stage_ev[k][i + 1]) for k in range(args.steps))
                 for i, n in enumerate(stage_names)}
 
-    launches_per_step = (4 + (1 if wl.max_entries > 16384 else 0)) if csa else 2
+    launches_per_step = decode_launches(wl)
     # ---- single-step latency: one step per replay of a one-step CUDA graph, the device idle before
     # it (synchronised between steps), events on the launching stream. This is what one decode step
     # of this layer costs on its own, without the overlap of consecutive steps' launches.

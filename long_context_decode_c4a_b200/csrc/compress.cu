@@ -312,6 +312,7 @@ __global__ void __cluster_dims__(kC128Split, 1, 1) __launch_bounds__(kCompressTh
   __shared__ float ss_w[CH / 8];
   __shared__ float ss_all[kC128Split];  // every CTA's partial sum of squares, written by that CTA
   const CompressParams& P = L.p[0];
+  cluster_arrive_relaxed();  // waited for before the first store into another CTA's shared memory
   timeline_mark(P.status, kTlCompress, kTlEntry);
   pdl_wait();
   pdl_trigger();
@@ -441,6 +442,7 @@ __global__ void __cluster_dims__(kC128Split, 1, 1) __launch_bounds__(kCompressTh
     if ((tid & 7) == 0) ss_w[tid >> 3] = sq;
   }
   __syncthreads();
+  cluster_wait();  // every CTA of the cluster has started: its shared memory may be written
   if (tid < kC128Split) {
     // Thread r stores this CTA's partial into slot `rank` of CTA r's ss_all.
     float v = 0.f;

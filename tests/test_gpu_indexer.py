@@ -84,6 +84,35 @@ def test_topk_two_stage_long_rows(ops):
         check_topk(idx[b, 0], ref, topk, f"b={b}")
 
 
+def test_topk_long_rows_exact(ops):
+    """Rows of 262144 entries (chunks of 16384 selected apart, then their lists merged): random
+    scores; one value everywhere (the first k indices); two values whose tie at the threshold spans
+    chunk boundaries; +-inf and NaN with a shorter visible count; and a row with fewer visible
+    entries than k. Exact against the oracle's selection on the same fp32 scores."""
+    B, E, k = 5, 262144, 1024
+    g = torch.Generator().manual_seed(23)
+    sc = torch.randn(B, 1, E, generator=g)
+    sc[1] = 0.5
+    sc[2] = 0.5
+    hot = torch.randperm(E, generator=g)[:500]
+    sc[2, 0, hot] = 1.0                                  # 500 above, the first 524 of the 0.5s kept
+    sc[3, 0, ::1001] = float("inf")
+    sc[3, 0, 7::2003] = float("nan")
+    sc[3, 0, 11::3001] = -float("inf")
+    pos = torch.full((B, 1), 4 * E - 1, dtype=torch.int32)
+    pos[3, 0] = 4 * 100000 - 1                          # 100000 visible entries
+    pos[4, 0] = 4 * 900 - 1                             # 900 visible entries < k
+    idx = ops.topk(pos.cuda(), sc.cuda(), k)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    for b in range(B):
+        Eb = min((int(pos[b, 0]) + 1) // 4, E)
+        want = O.topk_select(sc[b, 0, :Eb].double().numpy(), k)
+        assert np.array_equal(idx[b, 0], want), f"row {b}"
+    assert np.array_equal(idx[1, 0], np.arange(k))
+    assert np.array_equal(idx[4, 0], np.r_[np.arange(900), -np.ones(k - 900)])
+
+
 def test_topk_edge_cases(ops):
     """No visible entry, fewer entries than k, and exactly k entries."""
     B, S, H_I, topk = 1, 4, 64, 16
