@@ -816,20 +816,42 @@ __global__ void __launch_bounds__(kAttnCombineThreads) attn_combine_kernel(AttnC
   const int h = blockIdx.x, qi = blockIdx.y, dim = 4 * threadIdx.x;
   const int ns = P.splits;
   const long long item0 = (long long)qi * ns;
+  // Every split's max and denominator first (independent loads), then the partials four at a time,
+  // so the loads of a thread are in flight together rather than one latency each.
+  float ms[kAttnMaxSplits], ls[kAttnMaxSplits];
   float M = -CUDART_INF_F;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, P.part_ml[(item0 + s) * 2 * P.H + h]);
+#pragma unroll
+  for (int s = 0; s < kAttnMaxSplits; ++s) {
+    if (s < ns) {
+      const long long r = (item0 + s) * 2 * P.H + h;
+      ms[s] = P.part_ml[r];
+      ls[s] = P.part_ml[r + P.H];
+      M = fmaxf(M, ms[s]);
+    }
+  }
   float L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < ns; ++s) {
-    const long long r = (item0 + s) * 2 * P.H + h;
-    const float ms = P.part_ml[r], ls = P.part_ml[r + P.H];
-    const float w = ms == -CUDART_INF_F ? 0.f : exp2f(ms - M);
-    L += w * ls;
-    const float4 o = *reinterpret_cast<const float4*>(P.part_o + ((item0 + s) * P.H + h) * P.d + dim);
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
+  const float* po = P.part_o + (item0 * P.H + h) * P.d + dim;
+  const long long stride = (long long)P.H * P.d;  // from one split's row to the next's
+#pragma unroll
+  for (int s0 = 0; s0 < kAttnMaxSplits; s0 += 4) {
+    if (s0 >= ns) break;
+    float4 o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (s0 + u < ns) o[u] = *reinterpret_cast<const float4*>(po + (s0 + u) * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int s = s0 + u;
+      if (s < ns) {
+        const float w = ms[s] == -CUDART_INF_F ? 0.f : exp2f(ms[s] - M);
+        L += w * ls[s];
+        acc.x += w * o[u].x;
+        acc.y += w * o[u].y;
+        acc.z += w * o[u].z;
+        acc.w += w * o[u].w;
+      }
+    }
   }
   const float inv = 1.f / L;
   float y[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};

@@ -94,3 +94,14 @@ def test_graph_rounds_fit_the_timed_steps():
     for steps in range(1, 60):
         r = bench.graph_rounds(10, steps, 4)
         assert r >= 1 and (r * 4 <= steps or steps < 4)
+
+
+def test_decode_launch_counts_follow_the_library_rules():
+    """gpu_launches claims: CSA 32K = indexer (compressor step inside) + top-k + attention; 1M
+    context = indexer + top-k chunks + merge + attention split over 9 pairs per query + combine; HCA
+    = C128A step + attention; a small CSA batch splits its attention (combine added)."""
+    import bench
+    assert bench.decode_launches(WORKLOADS["pro_csa_decode_32k"]) == 3
+    assert bench.decode_launches(WORKLOADS["long_csa_decode_1m"]) == 5
+    assert bench.decode_launches(WORKLOADS["pro_hca_decode_32k"]) == 2
+    assert bench.decode_launches(WORKLOADS["pro_csa_decode_32k"].scaled(B=8)) == 4
