@@ -51,10 +51,16 @@ def load_peaks():
 
 
 def kernel_hash(files):
+    """Hash of the kernel's sources with comments and blank space removed: a recorded ncu capture
+    stays valid across comment edits and is invalidated by any change to the code."""
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "long_context_decode_c4a_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "long_context_decode_c4a_b200", "csrc", f), encoding="utf-8") as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        h.update(" ".join(src.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -30,11 +30,15 @@
 //     (one thread issues a tcgen05.mma only every ~50 cycles); 6 issues the PV MMAs in tile order
 //     (and owns TMEM); 7..10 load the partial scores of their 32 heads, free the score tile, stage
 //     the 4 KB in the outgoing buffer and bulk-copy it into the same quadrant's rows of the other
-//     CTA's incoming buffer; 11..14 add this CTA's staged partial scores and the other CTA's, run
-//     the softmax and store P. A sender and a softmax warp of the same TMEM lane quadrant trade
-//     with the two warps of that quadrant in the other CTA, with barriers of their own, so the four
-//     quadrants run independently. Warps 7..14 own one head (TMEM lane) per thread and share the
-//     epilogue.
+//     CTA's incoming buffer; 11..14 (even tiles) and 15..18 (odd tiles) add this CTA's staged
+//     partial scores and the other CTA's, run the softmax (the running max passes from one group to
+//     the other after every tile) and store P. A sender and the softmax warps of the same TMEM lane
+//     quadrant trade with the warps of that quadrant in the other CTA, with barriers of their own,
+//     so the four quadrants run independently. Warps 7..14 own one head (TMEM lane) per thread and
+//     share the epilogue.
+// Split-candidate mode (few queries): the pair of work item (query, split) takes one contiguous run
+// of the query's tiles and leaves its unnormalised O, max and denominator in the workspace;
+// attn_combine_kernel (end of this file) merges the splits.
 // Precision: P = P_hi + P_lo with both parts in bf16 (about 16 significant bits), accumulated by two
 // PV MMAs; a single bf16 P (8 bits) leaves errors near 1% of the output RMS on short candidate sets.
 // Online softmax in the log2 domain; the running max starts at the sink; O is rescaled only when a

@@ -10,11 +10,13 @@
 //   C128A (ratio 128): the 128 tokens of group g, one width-d stream.
 // then RMSNorm over the d channels and RoPE on the last rope_dim channels at position g*ratio.
 //
-// Two kernels. Decode (one token per request): compress_decode_kernel, one CTA per (request,
-// stream), feeds the token to the rolling state and pools the group it completes. Segments
-// (prefill): compress_kernel, one CTA per (request, completed group), each thread owning 8
-// consecutive channels read with 16-byte loads, then compress_state_kernel for the final state.
-// Memory-bound: no tensor-core work here.
+// Decode (one token per request): compress_decode_kernel, one CTA per (request, stream), feeds the
+// token to the rolling state and pools the group it completes (the fused CSA decode step runs the
+// same body inside the indexer launch); for C128A with d = 512, compress_decode_c128_kernel spreads
+// a request's 128 rows x 512 channels over a cluster of 8 channel-block CTAs. Segments (prefill):
+// compress_kernel, one CTA per (request, completed group), each thread owning 8 consecutive
+// channels read with 16-byte loads, then compress_state_kernel for the final state. Memory-bound:
+// no tensor-core work here.
 
 #include <cuda_bf16.h>
 #include <math_constants.h>
