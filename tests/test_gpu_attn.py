@@ -191,8 +191,9 @@ def test_split_candidates_match_one_pair_per_query(ops, mode, out_dtype):
         ref = O.attend_query(np64(q[b, 0]), t, W, np64(ring[b]), W, np64(cache[b]), sel, np64(sink),
                              1 / math.sqrt(d), 64, 10000.0)
         bf = out_dtype == torch.bfloat16
-        assert_attn_close(split[b, 0], ref, f"{mode} split b={b} t={t}", bf16_out=bf)
-        assert_attn_close(single[b, 0], ref, f"{mode} one pair b={b} t={t}", bf16_out=bf)
+        tag = f"{mode} {'bf16' if bf else 'fp32'} out"
+        assert_attn_close(split[b, 0], ref, f"{tag} split b={b} t={t}", bf16_out=bf)
+        assert_attn_close(single[b, 0], ref, f"{tag} one pair b={b} t={t}", bf16_out=bf)
     # The two differ only by rounding (other running maxima for P's bf16 parts, another order of the
     # same sums, and for bf16 output one rounding step): far below what a dropped or misweighted split
     # would leave.
