@@ -115,6 +115,46 @@ def test_decode_step_at_32k(ops):
             assert torch.count_nonzero(cache[b, :E - 1]) == 0
 
 
+@pytest.mark.parametrize("ratio", [4, 128])
+def test_decode_step_mixed_positions(ops, ratio):
+    """One decode step for requests at different positions: some complete a group in the step
+    (C128A: group 0 too), some do not; each request's entry and state against the oracle, and no
+    other cache row touched."""
+    d = 512
+    overlap = 1 if ratio == 4 else 0
+    width = (1 + overlap) * d
+    rows = (1 + overlap) * ratio
+    # C4A's group 0 has no previous group (its slots are the reset state's, weight 0), so a random
+    # state is a valid input there only for C128A.
+    pos = [32767, 32766, 127 if ratio == 128 else 7, 5000, 2 * ratio - 1]
+    B = len(pos)
+    g = torch.Generator().manual_seed(31 + ratio)
+    skv0 = torch.randn(B, rows, width, generator=g).to(torch.bfloat16)
+    ssc0 = torch.randn(B, rows, width, generator=g).to(torch.bfloat16)
+    kv = torch.randn(B, 1, width, generator=g).to(torch.bfloat16)
+    sc = torch.randn(B, 1, width, generator=g).to(torch.bfloat16)
+    gamma = (1 + 0.1 * torch.randn(d, generator=g)).to(torch.bfloat16)
+    E = 32768 // ratio
+    cache = torch.zeros(B, E, d, dtype=torch.bfloat16, device="cuda")
+    cache32 = torch.zeros(B, E, d, dtype=torch.float32, device="cuda")
+    skv, ssc = skv0.cuda(), ssc0.cuda()
+    ops.compress(ops.compressor_cfg(ratio, d), torch.tensor(pos, dtype=torch.int32, device="cuda"), kv.cuda(),
+                 sc.cuda(), gamma.cuda(), skv, ssc, cache, cache32)
+    torch.cuda.synchronize()
+    ocfg = O.CompressorCfg(ratio, d)
+    for b, t in enumerate(pos):
+        okv, osc = np64(skv0[b]).copy(), np64(ssc0[b]).copy()
+        res = O.compressor_step(ocfg, okv, osc, t, np64(kv[b, 0]), np64(sc[b, 0]), np64(gamma))
+        assert np.array_equal(np64(skv[b]), okv) and np.array_equal(np64(ssc[b]), osc), f"state b={b} t={t}"
+        touched = torch.nonzero(cache[b].abs().sum(-1)).flatten().tolist()
+        if (t + 1) % ratio == 0:
+            gi, entry = res
+            assert gi == t // ratio and touched == [gi], f"b={b} t={t}"
+            assert_compress_close(cache32[b, gi:gi + 1], cache[b, gi:gi + 1], entry[None], f"ratio {ratio} b={b} t={t}")
+        else:
+            assert res is None and touched == [], f"b={b} t={t}"
+
+
 def test_state_reset_values(ops):
     cfg = ops.compressor_cfg(4, 128)
     skv = torch.full((2, 8, 256), 3.0, dtype=torch.bfloat16, device="cuda")
