@@ -210,8 +210,22 @@ def decode_bytes(wl):
 
 def step_inputs(inp):
     keys = ["pos", "kv", "score", "idx_kv", "idx_score", "win_kv", "q", "q_idx", "w"]
-    return {k: inp[k][:, 0].contiguous() if inp[k].dim() > 1 and k != "pos" else inp[k][:, 0].contiguous()
-            for k in keys if k in inp}
+    return {k: inp[k][:, 0].contiguous() for k in keys if k in inp}
+
+
+def packed_layout(tensors, align: int = 256):
+    """Byte offsets of `tensors` laid end to end, each at a multiple of `align`, and the total size."""
+    offs, total = {}, 0
+    for k, v in tensors.items():
+        offs[k] = total
+        total += -(-v.numel() * v.element_size() // align) * align
+    return offs, total
+
+
+def packed_views(flat, tensors, offs):
+    """Views of the uint8 buffer `flat` with the dtype and shape of each of `tensors`."""
+    return {k: flat[offs[k]:offs[k] + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+            for k, v in tensors.items()}
 
 
 def run_ours_decode(wl, args, world, rank, light: bool = False):
@@ -355,12 +369,19 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
     # ---- end-to-end through the public API with host buffers: every step copies its inputs from
     # pinned host memory, runs, and copies its output back. Copies run on their own streams and
     # overlap the neighbouring steps' compute (two device buffer sets, events between streams).
+    # A step's inputs sit in one pinned host buffer (each at a 256-byte offset) and reach the device
+    # in one copy, into views of one device buffer that the prepared step reads.
     st, x = sets[0]
-    host = {k: v.to("cpu").pin_memory() for k, v in x.items() if k not in ("out", "sink")}
+    inputs = {k: v for k, v in x.items() if k not in ("out", "sink")}
+    offs, total = packed_layout(inputs)
+    host_flat = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for k, v in packed_views(host_flat, inputs, offs).items():
+        v.copy_(inputs[k])
     out_host = [torch.empty(x["out"].shape, dtype=x["out"].dtype).pin_memory() for _ in range(2)]
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    h2d = total
     d2h = out_host[0].numel() * out_host[0].element_size()
-    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host.items()} for _ in range(2)]
+    dev_flat = [torch.empty(total, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dev_in = [packed_views(f, inputs, offs) for f in dev_flat]
     dev_out = [torch.empty_like(x["out"]) for _ in range(2)]
     e2e_preps = []   # [buffer][input set]
     for buf in range(2):
@@ -388,8 +409,7 @@ def run_ours_decode(wl, args, world, rank, light: bool = False):
         buf = i % 2
         s_h2d.wait_event(comp_done[buf])          # step i-2 finished reading dev_in[buf]
         with torch.cuda.stream(s_h2d):
-            for k, v in host.items():
-                dev_in[buf][k].copy_(v, non_blocking=True)
+            dev_flat[buf].copy_(host_flat, non_blocking=True)
             h2d_done[buf].record(s_h2d)
         comp.wait_event(h2d_done[buf])
         comp.wait_event(d2h_done[buf])             # step i-2's output was copied out of dev_out[buf]

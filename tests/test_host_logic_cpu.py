@@ -105,3 +105,29 @@ def test_decode_launch_counts_follow_the_library_rules():
     assert bench.decode_launches(WORKLOADS["long_csa_decode_1m"]) == 5
     assert bench.decode_launches(WORKLOADS["pro_hca_decode_32k"]) == 2
     assert bench.decode_launches(WORKLOADS["pro_csa_decode_32k"].scaled(B=8)) == 4
+
+
+def test_packed_inputs_round_trip_every_tensor():
+    """The end-to-end timing copies a step's inputs in one buffer: every tensor of a decode step gets
+    its own 256-byte aligned, non-overlapping slot, and the views give back the same values."""
+    g = torch.Generator().manual_seed(5)
+    inputs = {
+        "pos": torch.randint(0, 1 << 20, (3,), dtype=torch.int32, generator=g),
+        "kv": torch.randn(3, 2, 512, generator=g),
+        "win_kv": torch.randn(3, 512, generator=g).to(torch.bfloat16),
+        "q": torch.randn(3, 5, 512, generator=g).to(torch.bfloat16),
+        "w": torch.randn(3, 7, generator=g),
+    }
+    offs, total = bench.packed_layout(inputs)
+    spans = sorted((offs[k], offs[k] + v.numel() * v.element_size()) for k, v in inputs.items())
+    assert all(o % 256 == 0 for o in offs.values())
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    assert total % 256 == 0 and spans[-1][1] <= total
+    flat = torch.zeros(total, dtype=torch.uint8)
+    views = bench.packed_views(flat, inputs, offs)
+    for k, v in views.items():
+        v.copy_(inputs[k])
+    again = bench.packed_views(flat.clone(), inputs, offs)
+    for k, v in inputs.items():
+        assert again[k].dtype == v.dtype and again[k].shape == v.shape
+        assert torch.equal(again[k], v), k
