@@ -177,6 +177,8 @@ CSA_API int csa_indexer_topk(int B, int S, int H_I, int d_I, int ratio, int topk
  *   out    dev [B, S, H, d]: bf16 if out_is_f32 == 0, float otherwise.
  * Supported: d = 512, rope_dim 64, 1 <= H <= 128, window <= 1024, topk <= 2048.
  * Alignment: pointers 16 bytes; ring_bstride and cache_bstride multiples of d.
+ * A selected index s >= min((t+1)//ratio, max_entries) (an entry not visible at t) is skipped and
+ * records CSA_ERR_BOUNDS in the workspace's status word (csa_get_device_status).
  */
 CSA_API int csa_sparse_attn(int B, int S, int H, int d, int rope_dim, float rope_base, float scale,
                     const int32_t* q_pos, const uint16_t* q, const uint16_t* ring,
@@ -188,7 +190,8 @@ CSA_API int csa_sparse_attn(int B, int S, int H, int d, int rope_dim, float rope
 /*
  * hca_attn -- HCA attention ([P5] §3: no index module): as csa_sparse_attn, but the compressed
  * candidates are every visible entry s < (t+1)//ratio (capped at max_entries), read in order.
- * Supported: as csa_sparse_attn, with at most 2048 visible entries per query.
+ * Supported: as csa_sparse_attn, with at most 2048 visible entries per query; a query with more
+ * attends to the first 2048 and records CSA_ERR_BOUNDS in the workspace's status word.
  */
 CSA_API int hca_attn(int B, int S, int H, int d, int rope_dim, float rope_base, float scale, int ratio,
              const int32_t* q_pos, const uint16_t* q, const uint16_t* ring, int64_t ring_bstride,

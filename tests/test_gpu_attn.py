@@ -200,3 +200,46 @@ def test_split_candidates_match_one_pair_per_query(ops, mode, out_dtype):
     rms = single.float().square().mean().sqrt()
     bound = 2e-3 * float(rms) + (float(single.float().abs().max()) * 2.0 ** -8 if out_dtype == torch.bfloat16 else 0.0)
     assert float((split.float() - single.float()).abs().max()) <= bound
+
+
+@pytest.mark.parametrize("mode", ["csa", "hca"])
+def test_largest_candidate_sets(ops, mode):
+    """The largest candidate set the attention takes: a window of 1024 rows plus 2048 selected (CSA)
+    or 2048 visible (HCA) entries, 96 tiles per query. Run with one CTA pair per query (the whole
+    list in one pair's shared memory) and with the tiles split over pairs; both match the oracle and
+    report no device error."""
+    from long_context_decode_c4a_b200 import _lib
+    g = torch.Generator().manual_seed(31)
+    B, S, H, d, W = 2, 1, 128, 512, 1024
+    if mode == "csa":
+        ratio, E_cap = 4, 12000
+        pos = torch.tensor([[40000], [8195]], dtype=torch.int32)   # 10000 and 2049 entries visible
+        topk = _random_topk(B, S, pos, 2048, ratio, g)
+    else:
+        ratio, E_cap = 128, 2048
+        pos = torch.tensor([[2048 * 128 + 100], [2048 * 128 - 1]], dtype=torch.int32)  # 2048 visible
+        topk = None
+    q = _q(B, S, H, d, g)
+    ring = torch.randn(B, W, d, generator=g).to(torch.bfloat16)
+    cache = torch.randn(B, E_cap, d, generator=g).to(torch.bfloat16)
+    sink = torch.randn(H, generator=g)
+    kind = _lib.CSA_WS_SPARSE_ATTN if mode == "csa" else _lib.CSA_WS_HCA_ATTN
+    refs = []
+    for b in range(B):
+        t = int(pos[b, 0])
+        sel = [int(s) for s in topk[b, 0] if s >= 0] if mode == "csa" else list(range(min((t + 1) // ratio, E_cap)))
+        assert len(sel) == 2048
+        refs.append(O.attend_query(np64(q[b, 0]), t, W, np64(ring[b]), W, np64(cache[b]), sel, np64(sink),
+                                   1 / math.sqrt(d), 64, 10000.0))
+    args = [x.cuda() for x in (pos, q, ring, cache)]
+    for label, ws in (("one pair", torch.zeros(256, dtype=torch.uint8, device="cuda")),
+                      ("split", ops.workspace(kind, B, S, 1, 1, "cuda"))):
+        out = torch.empty(B, S, H, d, dtype=torch.float32, device="cuda")
+        if mode == "csa":
+            ops.sparse_attn(*args, topk.cuda(), sink.cuda(), W, out=out, ws=ws)
+        else:
+            ops.hca_attn(*args, sink.cuda(), W, ratio=ratio, out=out, ws=ws)
+        torch.cuda.synchronize()
+        assert ops.device_status(ws) == _lib.CSA_OK, label
+        for b in range(B):
+            assert_attn_close(out[b, 0], refs[b], f"{mode} {label} b={b}")
