@@ -12,7 +12,6 @@ prefill segment to decode steps.
   each checked against the oracle's query at the same position over the whole token stream.
 """
 
-import ctypes
 import math
 
 import numpy as np

@@ -7,7 +7,6 @@ memory. This file is collected last so that a failure here leaves every other te
 it passes both alone in a fresh process and after the rest of the suite.
 """
 
-import ctypes
 import math
 
 import pytest
