@@ -407,6 +407,7 @@ struct AttnArgs {
   void* ws;
   size_t ws_bytes;
   size_t part_off = kStatusBytes;  // workspace offset of the split-candidate partials
+  bool early_window = false;       // q and the ring are final before the dependency wait (AttnParams)
 };
 
 // Split-candidate attention: a query's candidate tiles are spread over `splits` CTA pairs when the
@@ -481,6 +482,7 @@ int run_attn(const AttnArgs& a, bool csa_mode, cudaStream_t st) {
   P.status = reinterpret_cast<uint32_t*>(a.ws);
   P.ring = a.ring;
   P.cache = a.cache;
+  P.early_window = a.early_window ? 1 : 0;
   CUtensorMap map_q;
   const long long queries = (long long)a.B * a.S;
   if (int rc = make_map_2d(&map_q, a.q, 512, (uint64_t)queries * a.H, 512, 64, 128)) return rc;
@@ -877,6 +879,9 @@ int csa_decode_fused(const csa_decode_args* a, void* stream) {
   const IdxWs L = indexer_ws_layout(a->B, a->max_entries, a->topk, true);
   if (int rc = check_ws(a->ws, a->ws_bytes, L.total)) return rc;
   aa.part_off = L.total;  // the attention's split partials follow the indexer's buffers
+  // The ring row of token t is written by the indexer launch; the top-k launch between it and the
+  // attention waits for it to complete before it triggers the attention's launch.
+  aa.early_window = true;
 
   uint32_t* status = static_cast<uint32_t*>(a->ws);
   CompressLaunch CL{};

@@ -300,9 +300,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   timeline_mark(P.status, kTlAttn, kTlEntry);
-  pdl_wait();
-  pdl_trigger();
-  timeline_mark(P.status, kTlAttn, kTlReady);
+  // With early_window the producers wait for the previous launch only before they read the
+  // selection (below); every other warp waits here.
+  const bool early = P.early_window != 0;
+  if (!early || warp >= kProducers / 32) {
+    pdl_wait();
+    pdl_trigger();
+  }
+  if (!early) timeline_mark(P.status, kTlAttn, kTlReady);
   const int t = P.q_pos[qi];
   if (threadIdx.x == 0) trace_time(status, 0);
 
@@ -346,6 +351,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kAttnThreads, 1)
     named_bar_sync(2, kProducers);
     const int w_tiles = P.splits == 1 ? min(nwin / kTile, kStages) : 0;
     for (int tile = 0; tile < w_tiles; ++tile) issue(tile);
+    if (early) {
+      pdl_wait();   // the selection comes from the previous launch
+      pdl_trigger();
+      timeline_mark(P.status, kTlAttn, kTlReady);
+    }
     const int ecap = min((t + 1) / P.ratio, P.max_entries);
     int n = nwin;
     bool bad = false;

@@ -145,6 +145,11 @@ struct AttnParams {
   int splits;
   float* part_o;
   float* part_ml;
+  // Nonzero when q, q_pos and the ring rows are final before the kernel's dependency wait: the
+  // launch before this one waits for the launch that writes them before it lets this one start
+  // (the fused CSA decode step: compressor step and ring write in the indexer launch, then top-k,
+  // then this kernel). The producers then load Q and gather the window tiles first.
+  int early_window;
 };
 
 __global__ void attn_kernel(const __grid_constant__ CUtensorMap map_q, AttnParams P);
