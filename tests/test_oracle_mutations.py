@@ -6,8 +6,13 @@ written. The pins of test_oracle_pins.py then run against the mutant, and at lea
 fail. A control case runs the same pins against the unmodified source, which must pass them all, so a
 broken runner cannot pass for a caught mutant.
 
-Not listed, because no test can tell it apart from the oracle: dropping the +0.0 that folds -0
-into +0 before the top-k sort (numpy's sort already orders -0 and +0 as equal)."""
+Not listed, because no test can tell them apart from the oracle:
+- dropping the +0.0 that folds -0 into +0 before the top-k sort (numpy's sort already orders -0 and
+  +0 as equal);
+- writing C128A token t into state row (t + 1) % 128 instead of t % 128: the entry pools all 128
+  rows with one softmax, so any fixed permutation of the rows within a group gives the same entry.
+  Which row holds which token is a storage convention of the state (no page fixes it); the GPU
+  tests compare the kernels' state rows with the oracle's bit for bit."""
 
 import itertools
 import os
@@ -37,8 +42,18 @@ MUTATIONS = {
     "rmsnorm_without_eps": ("/ np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)",
                             "/ np.sqrt(np.mean(x * x, axis=-1, keepdims=True))"),
     "entry_visible_one_early": ("return (t + 1) // ratio", "return t // ratio + 1"),
+    "c4a_token_into_pre_rows": ("        row = r + t % r\n", "        row = t % r\n"),
+    "state_scores_not_rolled": ("        state_score[:r] = state_score[r:]\n", "        pass\n"),
+    "rmsnorm_without_gamma": ("return np.asarray(gamma, dtype=np.float64) * x / np.sqrt", "return x / np.sqrt"),
+    # rounding
+    "bf16_round_half_up": ("(((u >> np.uint64(16)) & np.uint64(1)) + np.uint64(0x7FFF))", "(np.uint64(0x8000))"),
+    "bf16_truncates": ("u = (u + (((u >> np.uint64(16)) & np.uint64(1)) + np.uint64(0x7FFF))) >> np.uint64(16)",
+                       "u = u >> np.uint64(16)"),
     # RoPE
     "rope_wrong_sign": ("y[..., head + 1::2] = even * s + odd * c", "y[..., head + 1::2] = -even * s + odd * c"),
+    "rope_frequency_exponent_halved": ("return float(pos) * np.power(float(base), -2.0 * i / rope_dim)",
+                                       "return float(pos) * np.power(float(base), -1.0 * i / rope_dim)"),
+    "rope_on_the_first_dims": ("    head = x.shape[-1] - rope_dim\n", "    head = 0\n"),
     # indexer and top-k
     "indexer_without_relu": ("return np.maximum(logits, 0.0) @", "return logits @"),
     "indexer_relu_after_weighting": (
@@ -47,8 +62,18 @@ MUTATIONS = {
     "ties_to_higher_index": ("order = np.lexsort((np.arange(n), -key, nan_last))",
                              "order = np.lexsort((-np.arange(n), -key, nan_last))"),
     "selection_in_score_order": ("sel = np.sort(order[: min(k, n)])", "sel = order[: min(k, n)]"),
+    "nan_sorts_highest": ("order = np.lexsort((np.arange(n), -key, nan_last))",
+                          "order = np.lexsort((np.arange(n), -key, -nan_last))"),
+    "indexer_scores_one_entry_too_many": ("k = np.asarray(idx_cache[:visible], dtype=np.float64)",
+                                          "k = np.asarray(idx_cache[:visible + 1], dtype=np.float64)"),
     # attention
     "window_shifted": ("return list(range(max(0, t - W + 1), t + 1))", "return list(range(max(0, t - W), t))"),
+    "window_ring_slot_off_by_one": ("rows = [ring[p % ring_cap] for p in window_positions(t, W)]",
+                                    "rows = [ring[(p + 1) % ring_cap] for p in window_positions(t, W)]"),
+    "padding_rows_gathered": ("rows += [cache[s] for s in selected if s >= 0]",
+                              "rows += [cache[s] for s in selected]"),
+    "sink_scaled_like_the_logits": ("m = np.maximum(np.max(logits, axis=1), sink)",
+                                    "sink = scale * sink\n    m = np.maximum(np.max(logits, axis=1), sink)"),
     "sink_left_out_of_the_max": ("m = np.maximum(np.max(logits, axis=1), sink)", "m = np.max(logits, axis=1)"),
     "sink_not_in_denominator": ("denom = np.sum(e, axis=1) + np.exp(sink - m)", "denom = np.sum(e, axis=1)"),
     "logits_unscaled": ("logits = scale * (q @ cand.T)", "logits = (q @ cand.T)"),
