@@ -89,6 +89,8 @@ MUTATIONS = {
                               "q = qraw / np.sqrt(np.mean(qraw * qraw, axis=(-2, -1), keepdims=True) + eps)"),
     "q_rotated_at_next_position": ("q[m] = rope(q[m], float(pos[m]), rope_dim, rope_base)",
                                    "q[m] = rope(q[m], float(pos[m]) + 1.0, rope_dim, rope_base)"),
+    "q_product_not_rounded": ("qraw = bf16(qr @ wq_b.T).reshape(M, H, d)", "qraw = (qr @ wq_b.T).reshape(M, H, d)"),
+    "window_row_not_rounded": ("w = bf16(x @ wkv.T)", "w = x @ wkv.T"),
     "window_row_not_rotated": (
         "return np.stack([rope(w[m], float(pos[m]), rope_dim, rope_base) for m in range(x.shape[0])])",
         "return w.copy()"),
@@ -105,6 +107,14 @@ MUTATIONS = {
     "hca_ring_written_after_attention": (
         'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, cache, list(range(vis)),',
         'out = attend_query(inp["q"][b, 0], t, W, inp["ring"][b], ring_cap, cache, list(range(vis)),'),
+    "decode_entry_not_rounded": ("        cache[g] = bf16(entry)\n    if res_idx", "        cache[g] = entry\n    if res_idx"),
+    "decode_index_stream_with_the_main_gamma": ('inp["idx_score"][b, 0], inp["idx_gamma"])',
+                                                'inp["idx_score"][b, 0], inp["gamma"])'),
+    "decode_in_step_entry_not_visible": ("    vis = visible_entries(t, ratio)\n    scores",
+                                         "    vis = visible_entries(t - 1, ratio)\n    scores"),
+    "hca_in_step_entry_not_visible": ("    vis = visible_entries(t, ratio)\n    out = attend_query",
+                                      "    vis = visible_entries(t - 1, ratio)\n    out = attend_query"),
+    "prefill_entries_not_rounded": ("    cache = bf16(entries)\n", "    cache = entries\n"),
     "hca_entry_written_after_attention": (
         'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, cache, list(range(vis)),',
         'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, inp["cache"][b], list(range(vis)),'),

@@ -522,6 +522,36 @@ def test_window_projection_one_hot_closed_form():
         assert np.allclose(w[m], _complex_rotate(x[m, sel], pos[m], 64, 10000.0), rtol=0, atol=1e-12)
 
 
+def test_q_path_rounds_the_product_before_the_head_norm():
+    """R21 on values fixed by hand: qa = [1, 1] gives qr = 1 / sqrt(1 + eps), which rounds to 1 in
+    bf16; Wq_b row 0 = [1, 2^-9] then gives 1 + 2^-9 in dim 0 of head 0 and every other row [1, 0]
+    gives 1. 1 + 2^-9 lies below half a bf16 step above 1, so the rounded product is 1 in every dim,
+    and the per-head norm leaves all unrotated dims of the head equal (1 / sqrt(1 + eps))."""
+    H, d, eps = 1, 512, 1e-6
+    x = np.array([[1.0, 1.0]])
+    wq_a = np.eye(2)
+    wq_b = np.zeros((H * d, 2))
+    wq_b[:, 0] = 1.0
+    wq_b[0, 1] = 2.0 ** -9
+    qa, qr, q = O.q_path(x, wq_a, np.ones(2), wq_b, np.array([0]), H, d, eps=eps)
+    assert np.array_equal(qr, np.ones((1, 2)))
+    want = 1.0 / np.sqrt(1.0 + eps)
+    assert np.all(q[0, 0, :d - 64] == want)
+
+
+def test_window_row_rounds_before_its_rotation():
+    """R21 on values fixed by hand: a window row whose dims 448 and 449 (the first rotated pair) come
+    out of the product as 1 + 2^-9 and 0 rounds to (1, 0) first, so at position 1 the pair is exactly
+    (cos theta_0, sin theta_0) = (cos 1, sin 1); an unrounded row would give (1 + 2^-9)(cos 1, sin 1)."""
+    d = 512
+    x = np.array([[1.0, 2.0 ** -9]])
+    wkv = np.zeros((d, 2))
+    wkv[448] = [1.0, 1.0]
+    w = O.window_projection(x, wkv, np.array([1]))
+    assert w[0, 448] == np.cos(1.0) and w[0, 449] == np.sin(1.0)
+    assert np.all(w[0, :448] == 0.0)
+
+
 # ----------------------------------------------------------------------------- decode step composition
 
 def _prefill_inputs(rng, S, H, d, ratio):
