@@ -35,6 +35,15 @@ MUTATIONS = {
     "direct_formula_wrong_half": (
         "slot_kv = np.concatenate([kv[prev, :d], kv[cur, d:]], axis=0)",
         "slot_kv = np.concatenate([kv[prev, d:], kv[cur, d:]], axis=0)"),
+    "first_group_takes_the_pre_channels": ("                slot_kv, slot_sc = kv[cur, d:], score[cur, d:]",
+                                           "                slot_kv, slot_sc = kv[cur, :d], score[cur, :d]"),
+    "fresh_state_scores_zero": ("    sc = np.full((cfg.state_rows, cfg.width), -np.inf)",
+                                "    sc = np.zeros((cfg.state_rows, cfg.width))"),
+    "pool_weights_from_kv": ("    e = np.where(valid, np.exp(np.where(valid, slot_score, 0.0) - m), 0.0)",
+                             "    e = np.where(valid, np.exp(np.where(valid, slot_kv, 0.0) - m), 0.0)"),
+    "segment_restarts_at_position_zero": (
+        "res = compressor_step(cfg, state_kv, state_score, start_pos + i, kv[i], score[i], gamma)",
+        "res = compressor_step(cfg, state_kv, state_score, i, kv[i], score[i], gamma)"),
     "state_not_rolled": ("        state_kv[:r] = state_kv[r:]\n", "        pass\n"),
     "softmax_over_channels": ("wts = e / np.sum(e, axis=0)", "wts = e / np.sum(e, axis=1, keepdims=True)"),
     "entry_position_off_by_one": ("rope(rms_norm(pooled, gamma, eps), g * ratio,",
@@ -51,6 +60,8 @@ MUTATIONS = {
                        "u = u >> np.uint64(16)"),
     # RoPE
     "rope_wrong_sign": ("y[..., head + 1::2] = even * s + odd * c", "y[..., head + 1::2] = -even * s + odd * c"),
+    "rope_inverse_ignored": ("    if inverse:\n        ang = -ang\n", "    if inverse:\n        pass\n"),
+    "rope_cos_sin_swapped": ("    c, s = np.cos(ang), np.sin(ang)", "    s, c = np.cos(ang), np.sin(ang)"),
     "rope_frequency_exponent_halved": ("return float(pos) * np.power(float(base), -2.0 * i / rope_dim)",
                                        "return float(pos) * np.power(float(base), -1.0 * i / rope_dim)"),
     "rope_on_the_first_dims": ("    head = x.shape[-1] - rope_dim\n", "    head = 0\n"),
@@ -62,6 +73,8 @@ MUTATIONS = {
     "ties_to_higher_index": ("order = np.lexsort((np.arange(n), -key, nan_last))",
                              "order = np.lexsort((-np.arange(n), -key, nan_last))"),
     "selection_in_score_order": ("sel = np.sort(order[: min(k, n)])", "sel = order[: min(k, n)]"),
+    "topk_takes_the_smallest": ("order = np.lexsort((np.arange(n), -key, nan_last))",
+                                "order = np.lexsort((np.arange(n), key, nan_last))"),
     "nan_sorts_highest": ("order = np.lexsort((np.arange(n), -key, nan_last))",
                           "order = np.lexsort((np.arange(n), -key, -nan_last))"),
     "indexer_scores_one_entry_too_many": ("k = np.asarray(idx_cache[:visible], dtype=np.float64)",
@@ -72,6 +85,10 @@ MUTATIONS = {
                                     "rows = [ring[(p + 1) % ring_cap] for p in window_positions(t, W)]"),
     "padding_rows_gathered": ("rows += [cache[s] for s in selected if s >= 0]",
                               "rows += [cache[s] for s in selected]"),
+    "one_max_over_all_heads": ("    m = np.maximum(np.max(logits, axis=1), sink)",
+                               "    m = np.maximum(np.max(logits, axis=0).max(), sink)"),
+    "hca_reads_capped_like_csa": ("return min(W, t + 1) + (vis if topk is None else min(topk, vis))",
+                                  "return min(W, t + 1) + (min(1024, vis) if topk is None else min(topk, vis))"),
     "sink_scaled_like_the_logits": ("m = np.maximum(np.max(logits, axis=1), sink)",
                                     "sink = scale * sink\n    m = np.maximum(np.max(logits, axis=1), sink)"),
     "sink_left_out_of_the_max": ("m = np.maximum(np.max(logits, axis=1), sink)", "m = np.max(logits, axis=1)"),
@@ -107,6 +124,9 @@ MUTATIONS = {
     "hca_ring_written_after_attention": (
         'out = attend_query(inp["q"][b, 0], t, W, ring, ring_cap, cache, list(range(vis)),',
         'out = attend_query(inp["q"][b, 0], t, W, inp["ring"][b], ring_cap, cache, list(range(vis)),'),
+    "decode_ring_slot_of_the_next_token": (
+        '    ring[t % ring_cap] = inp["win_kv"][b, 0]\n    vis = visible_entries(t, ratio)\n    scores',
+        '    ring[(t + 1) % ring_cap] = inp["win_kv"][b, 0]\n    vis = visible_entries(t, ratio)\n    scores'),
     "decode_entry_not_rounded": ("        cache[g] = bf16(entry)\n    if res_idx", "        cache[g] = entry\n    if res_idx"),
     "decode_index_stream_with_the_main_gamma": ('inp["idx_score"][b, 0], inp["idx_gamma"])',
                                                 'inp["idx_score"][b, 0], inp["gamma"])'),

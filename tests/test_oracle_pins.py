@@ -364,6 +364,18 @@ def test_reads_per_query_edge_cases():
     assert O.reads_per_query(1048575, 128, 4, 1024) == 1152
 
 
+def test_csa_and_hca_reads_cross_where_the_visible_entries_reach_k():
+    """[P1] "Pro 的 CSA 和 HCA，成本交点在哪里": top-k fixes CSA's reads (128 + 1024) while HCA reads
+    every visible entry, one per 128 tokens, so the two read counts are equal when (t + 1) / 128 =
+    1024, at a 128K context (t = 131071), and HCA reads more beyond it: 128 + 8192 at 1M."""
+    csa = lambda t: O.reads_per_query(t, 128, 4, 1024)
+    hca = lambda t: O.reads_per_query(t, 128, 128, None)
+    assert hca(32767) == 384 and csa(32767) == 1152
+    assert hca(131071) == csa(131071) == 1152
+    assert hca(131071 - 128) < csa(131071 - 128)
+    assert hca(1048575) == 128 + 8192 > csa(1048575)
+
+
 def test_prefill_totals_match_arithmetic_series():
     """An 8192-token CSA prefill from an empty cache, totalled over its queries and checked against
     sums of arithmetic series rather than a loop. u = t + 1 runs over 1..8192.
@@ -395,6 +407,25 @@ def test_large_sink_stays_finite():
     # = 0.3 e^-720 (a subnormal, about 2e-314), which an overflowed denominator would flush to 0.
     o = O.mqa_with_sink(q, c, np.array([720.4]), 1.0)
     assert np.allclose(o, 0.3 * math.exp(-720.0), rtol=1e-6, atol=0.0) and np.all(o > 0)
+
+
+def test_heads_have_softmaxes_of_their_own():
+    """[P5] §2.3 (MQA): the heads share one candidate set but each normalises its own logits, so a
+    head's output does not depend on the other heads, even when their logits lie 800 apart (far
+    beyond float64's exp range)."""
+    rng = np.random.default_rng(40)
+    cand = rng.standard_normal((6, 8))
+    cand[:, 0] = 1.0                     # a constant dim: q[h, 0] shifts every logit of head h
+    q = rng.standard_normal((3, 8))
+    q[1, 0] = 1000.0                     # head 1: logits near +1000
+    q[2, 0] = -1000.0                    # head 2: logits near -1000, far below its sink
+    sink = np.array([0.3, -1.0, 2.0])
+    together = O.mqa_with_sink(q, cand, sink, 1.0)
+    assert np.all(np.isfinite(together))
+    for h in range(3):
+        alone = O.mqa_with_sink(q[h:h + 1], cand, sink[h:h + 1], 1.0)
+        assert np.allclose(together[h], alone[0], rtol=1e-12, atol=1e-14)
+    assert np.allclose(together[2], 0.0, atol=1e-300)   # head 2: the sink takes all the weight
 
 
 def test_rmsnorm_eps_matters_for_small_vectors():
