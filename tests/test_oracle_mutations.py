@@ -12,7 +12,9 @@ Not listed, because no test can tell them apart from the oracle:
 - writing C128A token t into state row (t + 1) % 128 instead of t % 128: the entry pools all 128
   rows with one softmax, so any fixed permutation of the rows within a group gives the same entry.
   Which row holds which token is a storage convention of the state (no page fixes it); the GPU
-  tests compare the kernels' state rows with the oracle's bit for bit."""
+  tests compare the kernels' state rows with the oracle's bit for bit;
+- taking the slots' max over every slot instead of the valid ones: a missing slot's score is -inf,
+  which no max picks while one slot is valid."""
 
 import itertools
 import os
@@ -99,11 +101,19 @@ MUTATIONS = {
     # output projection
     "projection_wrong_group_weights": ('r = np.einsum("mgk,grk->mgr", og, wo_a)',
                                        'r = np.einsum("mgk,grk->mgr", og, wo_a[::-1])'),
+    "projection_groups_interleaved": ("    og = o_rows.reshape(M, G, Kg)\n",
+                                      "    og = o_rows.reshape(M, Kg, G).transpose(0, 2, 1)\n"),
     "projection_r_not_rounded": ("y = rb.reshape(M, G * R) @ wo_b.T", "y = r.reshape(M, G * R) @ wo_b.T"),
     # query path and window rows
     "q_without_gamma": ("qr = bf16(rms_norm(qa, gamma, eps))", "qr = bf16(rms_norm(qa, 1.0, eps))"),
     "q_norm_over_all_heads": ("q = qraw / np.sqrt(np.mean(qraw * qraw, axis=-1, keepdims=True) + eps)",
                               "q = qraw / np.sqrt(np.mean(qraw * qraw, axis=(-2, -1), keepdims=True) + eps)"),
+    "q_heads_split_wrong": ("qraw = bf16(qr @ wq_b.T).reshape(M, H, d)",
+                            "qraw = bf16(qr @ wq_b.T).reshape(M, d, H).transpose(0, 2, 1)"),
+    "q_head_norm_without_eps": ("q = qraw / np.sqrt(np.mean(qraw * qraw, axis=-1, keepdims=True) + eps)",
+                                "q = qraw / np.sqrt(np.mean(qraw * qraw, axis=-1, keepdims=True))"),
+    "window_row_rotated_at_next_position": ("rope(w[m], float(pos[m]), rope_dim, rope_base)",
+                                            "rope(w[m], float(pos[m]) + 1.0, rope_dim, rope_base)"),
     "q_rotated_at_next_position": ("q[m] = rope(q[m], float(pos[m]), rope_dim, rope_base)",
                                    "q[m] = rope(q[m], float(pos[m]) + 1.0, rope_dim, rope_base)"),
     "q_product_not_rounded": ("qraw = bf16(qr @ wq_b.T).reshape(M, H, d)", "qraw = (qr @ wq_b.T).reshape(M, H, d)"),
@@ -127,6 +137,11 @@ MUTATIONS = {
     "decode_ring_slot_of_the_next_token": (
         '    ring[t % ring_cap] = inp["win_kv"][b, 0]\n    vis = visible_entries(t, ratio)\n    scores',
         '    ring[(t + 1) % ring_cap] = inp["win_kv"][b, 0]\n    vis = visible_entries(t, ratio)\n    scores'),
+    "decode_scaled_by_the_index_width": (
+        '    scale = 1.0 / math.sqrt(d) if scale is None else scale\n    t = int(inp["pos"][b, 0])\n    main',
+        '    scale = 1.0 / math.sqrt(d_I) if scale is None else scale\n    t = int(inp["pos"][b, 0])\n    main'),
+    "hca_prefill_drops_the_last_entry": ("            scores, sel = None, np.arange(vis)",
+                                         "            scores, sel = None, np.arange(max(vis - 1, 0))"),
     "decode_entry_not_rounded": ("        cache[g] = bf16(entry)\n    if res_idx", "        cache[g] = entry\n    if res_idx"),
     "decode_index_stream_with_the_main_gamma": ('inp["idx_score"][b, 0], inp["idx_gamma"])',
                                                 'inp["idx_score"][b, 0], inp["gamma"])'),
